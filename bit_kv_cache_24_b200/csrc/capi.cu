@@ -1,0 +1,326 @@
+// capi.cu -- the C ABI declared in include/nvfp4.h: argument validation, layout arithmetic,
+// architecture checks and kernel dispatch.  No allocation, no synchronisation.
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace nvfp4 {
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+nvfp4_status cuda_fail(cudaError_t e, const char *where) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+    return NVFP4_ERR_CUDA;
+}
+
+struct DevInfo {
+    bool probed = false;
+    bool sm100 = false;
+    int sms = 148;
+};
+DevInfo g_dev[64];
+
+const DevInfo *device_info() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    DevInfo &d = g_dev[dev];
+    if (!d.probed) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return nullptr;
+        d.sm100 = (major == 10 && minor == 0);
+        d.sms = sms;
+        d.probed = true;
+    }
+    return &d;
+}
+
+// Common pre-flight: a usable sm_100 device is current.
+nvfp4_status check_device() {
+    const DevInfo *d = device_info();
+    if (!d) return cuda_fail(cudaGetLastError(), "device query");
+    if (!d->sm100) return NVFP4_ERR_UNSUPPORTED;
+    return NVFP4_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t codes_pitch(int64_t cols) { return 16 * ceil_div(cols, 32); }
+
+int64_t sf_bytes(int64_t rows, int64_t cols, int32_t layout) {
+    if (rows < 0 || cols < 0) return -1;
+    const int64_t nb = ceil_div(cols, 16);
+    if (layout == NVFP4_SF_LINEAR) return rows * nb;
+    if (layout == NVFP4_SF_MMA) return 128 * ceil_div(rows, 128) * 4 * ceil_div(nb, 4);
+    return -1;
+}
+
+}  // namespace
+
+int num_sms() {
+    const DevInfo *d = device_info();
+    return d ? d->sms : 148;
+}
+
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" {
+
+int32_t nvfp4_version(void) { return 100; }
+
+const char *nvfp4_last_error(void) { return g_last_error; }
+
+const char *nvfp4_status_string(int32_t status) {
+    switch (status) {
+        case NVFP4_OK: return "ok";
+        case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+        case NVFP4_ERR_UNSUPPORTED: return "unsupported shape, alignment, layout or architecture";
+        case NVFP4_ERR_NONFINITE: return "non-finite input";
+        case NVFP4_ERR_TIMEOUT: return "bounded on-chip wait timed out";
+        case NVFP4_ERR_CUDA: return "CUDA error";
+        default: return "unknown status";
+    }
+}
+
+int64_t nvfp4_codes_pitch(int64_t cols) { return cols < 0 ? -1 : codes_pitch(cols); }
+
+int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols, int32_t layout) { return sf_bytes(rows, cols, layout); }
+
+size_t nvfp4_quantize_workspace(int64_t rows, int64_t cols) {
+    (void)rows;
+    (void)cols;
+    return (size_t)kMaxPartials * sizeof(uint32_t);
+}
+
+size_t nvfp4_kv_append_workspace(int64_t ntok, int32_t heads, int32_t head_dim) {
+    (void)ntok;
+    (void)heads;
+    (void)head_dim;
+    return 2 * (size_t)kMaxPartials * sizeof(uint32_t);
+}
+
+nvfp4_status nvfp4_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ld, float *amax_out, void *ws,
+                        size_t ws_bytes, int32_t *dev_status, nvfp4_stream stream) {
+    if (!x_bf16 || !amax_out || !ws || M < 0 || K < 0 || ld < K) return NVFP4_ERR_INVALID_ARG;
+    if (ws_bytes < nvfp4_quantize_workspace(M, K)) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || !aligned16(ws) || (ld & 7) || (K & 7)) return NVFP4_ERR_UNSUPPORTED;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    RowJobs jobs{};
+    jobs.njobs = 1;
+    jobs.npartial = amax_blocks(M);
+    jobs.job[0].x = static_cast<const uint16_t *>(x_bf16);
+    jobs.job[0].rows = M;
+    jobs.job[0].cols = K;
+    jobs.job[0].ld = ld;
+    jobs.job[0].partial = static_cast<uint32_t *>(ws);
+    cudaError_t e = launch_amax(jobs, dev_status, amax_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_amax");
+}
+
+nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld, int32_t dir,
+                            const float *amax_in, const nvfp4_tensor *out, void *ws, size_t ws_bytes,
+                            int32_t *dev_status, nvfp4_stream stream) {
+    if (!x_bf16 || !out || !out->codes || !out->sf || !out->g || M <= 0 || K <= 0 || ld < K)
+        return NVFP4_ERR_INVALID_ARG;
+    if (dir != NVFP4_ROWWISE && dir != NVFP4_COLWISE) return NVFP4_ERR_INVALID_ARG;
+    if (out->sf_layout != NVFP4_SF_LINEAR && out->sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_INVALID_ARG;
+    const int64_t orows = dir == NVFP4_ROWWISE ? M : K, ocols = dir == NVFP4_ROWWISE ? K : M;
+    if (out->rows != orows || out->cols != ocols) return NVFP4_ERR_INVALID_ARG;
+    if (!amax_in && (!ws || ws_bytes < nvfp4_quantize_workspace(M, K))) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || (ld & 7) || (K & 7)) return NVFP4_ERR_UNSUPPORTED;
+    if (dir == NVFP4_ROWWISE && (K & 15)) return NVFP4_ERR_UNSUPPORTED;
+    if (!aligned16(out->codes) || (ws && !aligned16(ws))) return NVFP4_ERR_UNSUPPORTED;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    RowJobs jobs{};
+    jobs.njobs = 1;
+    jobs.npartial = amax_blocks(M);
+    RowJob &j = jobs.job[0];
+    j.x = static_cast<const uint16_t *>(x_bf16);
+    j.rows = M;
+    j.cols = K;
+    j.ld = ld;
+    j.codes = out->codes;
+    j.pitch = codes_pitch(ocols);
+    j.sf = out->sf;
+    j.sf_layout = out->sf_layout;
+    j.g_out = out->g;
+    j.amax_in = amax_in;
+    j.partial = static_cast<uint32_t *>(ws);
+    cudaError_t e = cudaSuccess;
+    if (!amax_in) e = launch_amax(jobs, dev_status, nullptr, s);
+    if (e == cudaSuccess) {
+        if (dir == NVFP4_ROWWISE) {
+            e = launch_quantize_rows(jobs, dev_status, s);
+        } else {
+            RowJob jc = j;
+            e = launch_quantize_cols(jc, jobs.npartial, dev_status, s);
+        }
+    }
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_quantize");
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16,
+                        const void *resid_bf16, void *y, int64_t ldy, int32_t y_dtype, int32_t *dev_status,
+                        nvfp4_stream stream) {
+    if (!A || !B || !y || !A->codes || !B->codes || !A->sf || !B->sf || !A->g || !B->g)
+        return NVFP4_ERR_INVALID_ARG;
+    if (A->rows <= 0 || B->rows <= 0 || A->cols <= 0 || A->cols != B->cols) return NVFP4_ERR_INVALID_ARG;
+    if (bias_bf16 && resid_bf16) return NVFP4_ERR_INVALID_ARG;
+    if (y_dtype != NVFP4_OUT_BF16 && y_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+    if (ldy < B->rows) return NVFP4_ERR_INVALID_ARG;
+    if (A->sf_layout != NVFP4_SF_MMA || B->sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_UNSUPPORTED;
+    if ((B->rows & 7) || (ldy & 7)) return NVFP4_ERR_UNSUPPORTED;
+    if (!aligned16(A->codes) || !aligned16(B->codes) || !aligned16(A->sf) || !aligned16(B->sf) || !aligned16(y))
+        return NVFP4_ERR_UNSUPPORTED;
+    if ((bias_bf16 && !aligned16(bias_bf16)) || (resid_bf16 && !aligned16(resid_bf16))) return NVFP4_ERR_UNSUPPORTED;
+    if ((A->rows + 127) / 128 > 0x7FFFFFFF / 128) return NVFP4_ERR_UNSUPPORTED;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    GemmArgs a{};
+    a.a_codes = A->codes;
+    a.b_codes = B->codes;
+    a.a_sf = A->sf;
+    a.b_sf = B->sf;
+    a.ga = A->g;
+    a.gb = B->g;
+    a.M = A->rows;
+    a.N = B->rows;
+    a.K = A->cols;
+    a.a_pitch = codes_pitch(A->cols);
+    a.b_pitch = codes_pitch(B->cols);
+    a.bias = static_cast<const uint16_t *>(bias_bf16);
+    a.resid = static_cast<const uint16_t *>(resid_bf16);
+    a.y = y;
+    a.ldy = ldy;
+    a.y_f32 = y_dtype == NVFP4_OUT_F32;
+    a.status = dev_status;
+    cudaError_t e = launch_gemm(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_gemm");
+}
+
+int64_t nvfp4_kv_cache_bytes(int32_t layers, int32_t heads, int32_t head_dim, int32_t slots, int32_t slot_tokens,
+                             int32_t which) {
+    if (layers <= 0 || heads <= 0 || head_dim <= 0 || slots <= 0 || slot_tokens <= 0) return -1;
+    const int64_t row = (int64_t)heads * head_dim, n = (int64_t)layers * slots;
+    switch (which) {
+        case 0: return n * slot_tokens * (row / 2);
+        case 1: return n * slot_tokens * (row / 16);
+        case 2: return n * (int64_t)sizeof(float);
+        default: return -1;
+    }
+}
+
+static bool kv_ok(const nvfp4_kv_cache *c) {
+    if (!c || c->layers <= 0 || c->heads <= 0 || c->head_dim <= 0 || c->slots <= 0 || c->slot_tokens <= 0) return false;
+    if (!c->codes_k || !c->codes_v || !c->sf_k || !c->sf_v || !c->g_k || !c->g_v || !c->len) return false;
+    return true;
+}
+
+nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int32_t slot, const void *k_bf16,
+                             const void *v_bf16, int64_t ntok, int64_t ld, void *ws, size_t ws_bytes,
+                             int32_t *dev_status, nvfp4_stream stream) {
+    if (!kv_ok(cache) || !k_bf16 || !v_bf16 || !ws) return NVFP4_ERR_INVALID_ARG;
+    if (layer < 0 || layer >= cache->layers || slot < 0 || slot >= cache->slots) return NVFP4_ERR_INVALID_ARG;
+    const int64_t row = (int64_t)cache->heads * cache->head_dim;
+    if (ntok <= 0 || ntok > cache->slot_tokens || ld < row) return NVFP4_ERR_INVALID_ARG;
+    if (ws_bytes < nvfp4_kv_append_workspace(ntok, cache->heads, cache->head_dim)) return NVFP4_ERR_INVALID_ARG;
+    if ((cache->head_dim & 15) || (row & 31) || (ld & 7)) return NVFP4_ERR_UNSUPPORTED;
+    if (!aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(ws) || !aligned16(cache->codes_k) ||
+        !aligned16(cache->codes_v))
+        return NVFP4_ERR_UNSUPPORTED;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    const int64_t slot_index = (int64_t)layer * cache->slots + slot;
+    const int64_t tok0 = slot_index * cache->slot_tokens;
+    RowJobs jobs{};
+    jobs.njobs = 2;
+    jobs.npartial = amax_blocks(ntok);
+    for (int i = 0; i < 2; ++i) {
+        RowJob &j = jobs.job[i];
+        j.x = static_cast<const uint16_t *>(i == 0 ? k_bf16 : v_bf16);
+        j.rows = ntok;
+        j.cols = row;
+        j.ld = ld;
+        j.codes = (i == 0 ? cache->codes_k : cache->codes_v) + tok0 * (row / 2);
+        j.pitch = row / 2;
+        j.sf = (i == 0 ? cache->sf_k : cache->sf_v) + tok0 * (row / 16);
+        j.sf_layout = NVFP4_SF_LINEAR;
+        j.g_out = (i == 0 ? cache->g_k : cache->g_v) + slot_index;
+        j.amax_in = nullptr;
+        j.partial = static_cast<uint32_t *>(ws) + i * kMaxPartials;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_amax(jobs, dev_status, nullptr, s);
+    if (e == cudaSuccess) e = launch_quantize_rows(jobs, dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "kv_quant_append");
+    cache->len[slot_index] = (int32_t)ntok;
+    return NVFP4_OK;
+}
+
+nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, const int32_t *slots, int32_t nslots,
+                        void *k_out_bf16, void *v_out_bf16, int32_t *dev_status, nvfp4_stream stream) {
+    if (!kv_ok(cache) || !slots || !k_out_bf16 || !v_out_bf16) return NVFP4_ERR_INVALID_ARG;
+    if (layer < 0 || layer >= cache->layers || nslots <= 0 || nslots > kMaxDequantSlots) return NVFP4_ERR_INVALID_ARG;
+    const int64_t row = (int64_t)cache->heads * cache->head_dim;
+    if ((cache->head_dim & 15) || (row & 31)) return NVFP4_ERR_UNSUPPORTED;
+    if (!aligned16(k_out_bf16) || !aligned16(v_out_bf16)) return NVFP4_ERR_UNSUPPORTED;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    static thread_local DequantJob jk, jv;
+    int64_t tok = 0;
+    int32_t n = 0;
+    for (int32_t i = 0; i < nslots; ++i) {
+        const int32_t s = slots[i];
+        if (s < 0 || s >= cache->slots) return NVFP4_ERR_INVALID_ARG;
+        const int64_t slot_index = (int64_t)layer * cache->slots + s;
+        const int32_t len = cache->len[slot_index];
+        if (len < 0 || len > cache->slot_tokens) return NVFP4_ERR_INVALID_ARG;
+        if (len == 0) continue;
+        const int64_t tok0 = slot_index * cache->slot_tokens;
+        jk.slot[n] = DequantSlot{cache->codes_k + tok0 * (row / 2), cache->sf_k + tok0 * (row / 16),
+                                 cache->g_k + slot_index, tok};
+        jv.slot[n] = DequantSlot{cache->codes_v + tok0 * (row / 2), cache->sf_v + tok0 * (row / 16),
+                                 cache->g_v + slot_index, tok};
+        tok += len;
+        ++n;
+    }
+    if (n == 0) return NVFP4_OK;
+    jk.nslots = jv.nslots = n;
+    jk.total_tokens = jv.total_tokens = tok;
+    jk.row_elems = jv.row_elems = row;
+    jk.out = static_cast<uint16_t *>(k_out_bf16);
+    jv.out = static_cast<uint16_t *>(v_out_bf16);
+    cudaError_t e = launch_kv_dequant(&jk, &jv, dev_status, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "kv_dequant");
+}
+
+nvfp4_status nvfp4_encode_elements(const float *in, int64_t n, uint8_t *e2m1_out, uint8_t *e4m3_out,
+                                   nvfp4_stream stream) {
+    if (!in || n < 0) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    cudaError_t e = launch_encode_elements(in, n, e2m1_out, e4m3_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_encode_elements");
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(int32_t *dev_status, int64_t limit_ns, nvfp4_stream stream) {
+    if (!dev_status || limit_ns <= 0 || limit_ns > 10000000000ll) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    cudaError_t e = launch_wait_timeout(dev_status, limit_ns, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_selftest_wait_timeout");
+}
+
+}  // extern "C"

@@ -1,0 +1,200 @@
+// common.cuh -- device helpers shared by the NVFP4 kernels (sm_100a only).
+//
+// Number formats follow the published NVFP4 format (E2M1 codes, E4M3 block scales, FP32 tensor
+// scale; round to nearest even, saturating).  The element and scale encoders use the Blackwell
+// hardware conversions (cvt.rn.satfinite.e2m1x2.f32 / e4m3x2.f32); decoders use the matching
+// cvt.rn.f16x2.{e2m1x2,e4m3x2}.  All FP32 arithmetic that decides a code is written with the
+// explicitly rounded intrinsics (__fdiv_rn, __frcp_rn, __fmul_rn) so that no contraction or
+// approximation can change a code.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/nvfp4.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ != 1000)
+#error "this library is written for sm_100a only"
+#endif
+
+namespace nvfp4 {
+
+constexpr float kE2M1Max = 6.0f;
+constexpr float kE4M3Max = 448.0f;
+constexpr float kGlobalDen = kE2M1Max * kE4M3Max;   // 2688: maps the tensor max to both grid tops
+
+// ---- status word ------------------------------------------------------------------------------
+
+__device__ __forceinline__ void set_status(int32_t *st, int32_t code) {
+    if (st) atomicCAS(st, 0, code);
+}
+
+// ---- conversions ------------------------------------------------------------------------------
+
+// Eight FP32 -> 32 bits of packed E2M1 codes, element 0 in the lowest nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const float q[8]) {
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+    return out;
+}
+
+// FP32 -> E4M3 byte (round to nearest even, saturating to +-448).
+__device__ __forceinline__ uint32_t e4m3(float v) {
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(v));
+    return out & 0xFFu;
+}
+
+// E4M3 byte -> FP32 (exact).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+    uint32_t h2;
+    uint16_t in = (uint16_t)(b & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Four bytes of packed E2M1 codes -> four f16x2 words (exact); element 2i in the low half of
+// out[i].
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t codes, uint32_t out[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(out[0]), "=r"(out[1]), "=r"(out[2]), "=r"(out[3]) : "r"(codes));
+}
+
+// Two FP32 -> packed BF16x2 (round to nearest even); `lo` in the low half.
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+    uint32_t out;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(out) : "f"(hi), "f"(lo));
+    return out;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Per-tensor decode scale from amax (FP32 IEEE division).
+__device__ __forceinline__ float global_scale(float amax) {
+    return amax == 0.0f ? 1.0f : __fdiv_rn(amax, kGlobalDen);
+}
+
+// ---- the 16-block quantization step -----------------------------------------------------------
+//
+// Given the block max b (exact BF16 value), g and den = g*6: the scale byte, and r = 1/d
+// (0 when d == 0, meaning every code of the block is +0).
+struct BlockScale {
+    uint32_t sf;
+    float r;
+    bool r_inf;   // d so small that 1/d overflows: x*r is then +-inf (or NaN for x == 0)
+};
+
+__device__ __forceinline__ BlockScale block_scale(float b, float g, float den) {
+    BlockScale s;
+    s.sf = (b == 0.0f) ? 0u : e4m3(__fdiv_rn(b, den));
+    const float d = __fmul_rn(e4m3_to_f32(s.sf), g);
+    s.r = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+    s.r_inf = isinf(s.r);
+    return s;
+}
+
+// Eight BF16 (as 4 packed words) -> 8 E2M1 codes given the block's reciprocal scale.
+// q = x*r in FP32 (IEEE RN); when r overflowed, zero inputs give +0 (their product would be
+// NaN, which encodes as +0) and the rest saturate.
+__device__ __forceinline__ uint32_t encode8(const uint32_t w[4], const BlockScale &s) {
+    float q[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        q[2 * i] = __fmul_rn(bf16_lo(w[i]), s.r);
+        q[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), s.r);
+    }
+    if (s.r_inf) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (bf16_lo(w[i]) == 0.0f) q[2 * i] = 0.0f;
+            if (bf16_hi(w[i]) == 0.0f) q[2 * i + 1] = 0.0f;
+        }
+    }
+    return e2m1x8(q);
+}
+
+// Max of |x| over 8 BF16 in 4 words, as BF16 magnitude bits (monotone in the magnitude).
+__device__ __forceinline__ uint32_t absmax_bits8(const uint32_t w[4]) {
+    uint32_t m = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
+    m = __vmaxu2(m, __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
+    return max(m & 0xFFFFu, m >> 16);
+}
+
+// ---- tensor-core scale layout -----------------------------------------------------------------
+
+// Byte offset of scale (row i, 16-block b) in the 128x4-atom tcgen05 block-scaling layout.
+__host__ __device__ __forceinline__ int64_t sf_mma_offset(int64_t i, int64_t b, int64_t atoms_per_row) {
+    return ((i >> 7) * atoms_per_row + (b >> 2)) * 512 + (i & 31) * 16 + ((i & 127) >> 5) * 4 + (b & 3);
+}
+
+__host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---- bounded waits ----------------------------------------------------------------------------
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+    return done != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after limit_ns or when *abort is raised.
+// Returns false when it gave up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  const volatile int *abort, uint64_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (abort && *abort) return false;
+            if (globaltimer_ns() - t0 > limit_ns) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbarrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s: far beyond any legitimate wait
+
+}  // namespace nvfp4

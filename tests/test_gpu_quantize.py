@@ -1,0 +1,116 @@
+"""GPU parity of nvfp4_amax / nvfp4_quantize (row-wise and column-wise, both scale layouts)
+against the CPU oracle: codes, scales and g must match bit for bit, padding included.
+Shapes span several tiles with ragged tails, the degenerate cases (zero tensor, one row, a
+partial 16-block, tiny magnitudes where 1/d overflows, inf/NaN input) and the full-size tensors
+of the DiT workloads."""
+import numpy as np
+import pytest
+import torch
+
+import bit_kv_cache_24_b200 as nv
+from bit_kv_cache_24_b200 import synth
+from tests.parity_util import assert_quantized_equal
+
+pytestmark = pytest.mark.gpu
+
+ROW_CASES = [(1, 16, "normal"), (3, 32, "outliers"), (128, 256, "outliers"), (130, 80, "wide"),
+             (257, 3072, "lognormal"), (1000, 1008, "wide"), (4680, 3072, "lognormal")]
+COL_CASES = [(16, 32, "normal"), (40, 24, "outliers"), (37, 8, "wide"), (300, 96, "lognormal"),
+             (4680, 256, "wide"), (1040, 136, "normal")]
+
+
+@pytest.mark.parametrize("layout", [nv.SF_LINEAR, nv.SF_MMA])
+@pytest.mark.parametrize("rows,cols,kind", ROW_CASES)
+def test_rowwise(orc, rows, cols, kind, layout):
+    x = synth.ragged(rows + cols, rows, cols, kind)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gq = nv.nvfp4_quantize(x.cuda(), nv.ROWWISE, sf_layout=layout, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    ost, oq = orc.quantize(x)
+    assert ost == 0
+    assert_quantized_equal(orc, gq, oq, f"row {rows}x{cols} {kind}")
+
+
+@pytest.mark.parametrize("layout", [nv.SF_LINEAR, nv.SF_MMA])
+@pytest.mark.parametrize("rows,cols,kind", COL_CASES)
+def test_colwise(orc, rows, cols, kind, layout):
+    x = synth.ragged(rows * 3 + cols, rows, cols, kind)
+    gq = nv.nvfp4_quantize(x.cuda(), nv.COLWISE, sf_layout=layout)
+    ost, oq = orc.quantize(x, colwise=True)
+    assert ost == 0
+    assert_quantized_equal(orc, gq, oq, f"col {rows}x{cols} {kind}")
+
+
+def test_strided_rows_and_amax_in(orc):
+    big = synth.ragged(5, 300, 1024, "lognormal")
+    x = big.cuda()[:, 128:640]                          # ld = 1024, K = 512
+    amax = nv.nvfp4_amax(x)
+    ref_st, ref_amax = orc.amax(big[:, 128:640].contiguous())
+    assert amax.item() == np.float32(ref_amax)
+    g1 = nv.nvfp4_quantize(x, nv.ROWWISE)
+    g2 = nv.nvfp4_quantize(x, nv.ROWWISE, amax_in=amax)
+    g3 = nv.nvfp4_quantize(x, nv.COLWISE, amax_in=amax)
+    _, o1 = orc.quantize(big[:, 128:640].contiguous())
+    _, o3 = orc.quantize(big[:, 128:640].contiguous(), colwise=True)
+    assert_quantized_equal(orc, g1, o1, "strided")
+    assert_quantized_equal(orc, g2, o1, "amax_in")
+    assert_quantized_equal(orc, g3, o3, "colwise amax_in")
+
+
+def test_zero_tensor(orc):
+    x = torch.zeros(64, 96, dtype=torch.bfloat16)
+    gq = nv.nvfp4_quantize(x.cuda(), nv.ROWWISE)
+    _, oq = orc.quantize(x)
+    assert_quantized_equal(orc, gq, oq, "zeros")
+    assert gq.g.item() == 1.0
+
+
+def test_tiny_magnitudes_where_reciprocal_overflows(orc):
+    # BF16 subnormal-range inputs: g and d are so small that 1/d overflows to inf; the zero
+    # elements then encode as +0 (their product would be NaN)
+    a = np.zeros((4, 64), np.float32)
+    a[0, :8] = 1e-39
+    a[1, 3] = -3e-40
+    a[2, ::3] = 2e-38
+    a[3, 1] = 1e-30
+    x = torch.from_numpy(a).to(torch.bfloat16)
+    gq = nv.nvfp4_quantize(x.cuda(), nv.ROWWISE, sf_layout=nv.SF_LINEAR)
+    _, oq = orc.quantize(x)
+    assert_quantized_equal(orc, gq, oq, "tiny")
+
+
+@pytest.mark.parametrize("bad", [float("inf"), float("nan")])
+def test_nonfinite_input_sets_status(bad):
+    x = torch.randn(64, 64).to(torch.bfloat16)
+    x[17, 5] = bad
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_quantize(x.cuda(), nv.ROWWISE, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == nv.NVFP4_ERR_NONFINITE
+    st.zero_()
+    nv.nvfp4_quantize(x.cuda(), nv.COLWISE, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == nv.NVFP4_ERR_NONFINITE
+
+
+def test_full_size_training_operands(orc):
+    """Training workload at full size: X [37440 x 3072] row-wise and column-wise (the wgrad
+    operand), every byte compared."""
+    X = synth.train()["X"]
+    xg = X.cuda()
+    amax = nv.nvfp4_amax(xg)
+    gr = nv.nvfp4_quantize(xg, nv.ROWWISE, amax_in=amax)
+    gc = nv.nvfp4_quantize(xg, nv.COLWISE, amax_in=amax)
+    _, orow = orc.quantize(X)
+    assert_quantized_equal(orc, gr, orow, "train X row")
+    del orow
+    _, ocol = orc.quantize(X, colwise=True)
+    assert_quantized_equal(orc, gc, ocol, "train X col")
+
+
+def test_full_size_ffn_down_activation(orc):
+    A = synth.ffn()["A_down"]                           # GELU output [4680 x 14336]
+    gq = nv.nvfp4_quantize(A.cuda(), nv.ROWWISE)
+    _, oq = orc.quantize(A)
+    assert_quantized_equal(orc, gq, oq, "ffn down A")
