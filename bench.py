@@ -1,0 +1,452 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 hot path on B200: one step = one autoregressive chunk through the QKV
+projection of a 5B-class video DiT layer with every NVFP4 operation of the path:
+
+  a4  weight quantize        W [9216 x 3072] BF16 -> NVFP4 (re-quantized each step, as in training)
+  a1  activation amax        A [4680 x 3072] (3 latent frames x 30 x 52 patches)
+  a2  row-wise quantize      A -> GEMM operand (amax reused)
+  a3  column-wise quantize   A -> token-dim blocks (the wgrad operand; amax reused)
+  a5+a6 NVFP4 GEMM + bias    Y [4680 x 9216] = gA*gB * A.W^T + bias, BF16
+  a7  KV append              K = Y[:, 3072:6144], V = Y[:, 6144:] (strided) -> cache slot (in place)
+  a8  KV restore             the 12-slot window (56160 tokens, 24 heads x 128) -> BF16 K and V
+
+`value` = NVFP4 GEMM FLOPs per step / device time per step (TFLOP/s), summed over ranks; the
+per-kernel throughputs and roofline fractions are in `kernels`, the dominant kernel's in
+`roofline`.  Inputs rotate over three input sets (~300 MB) and each step streams ~1.1 GB, so no
+step finds its inputs in the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica (the path has no exchange step);
+timing is the max over ranks of the device time.  `--impl reference` times the CPU oracle on a
+bounded row sample of the same step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 GEMM TFLOP/s (% FP4 peak); quantize/KV-dequant GB/s (% HBM peak)"
+UNIT = "TFLOP/s"
+M_TOK, HID, NQKV = 4680, 3072, 9216
+HEADS, HEAD_DIM, SLOTS = 24, 128, 12
+GEMM_FLOP = 2.0 * M_TOK * NQKV * HID
+FP4_OVER_BF16 = 9.0 / 2.25          # nominal dense FP4 : BF16 tensor throughput on B200
+PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=3000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--e2e-steps", type=int, default=40)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=15.0)
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------- plumbing
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def init_dist(world, backend):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def reduce_max(value: float, dist, device) -> float:
+    """Max over ranks of a per-rank time (timing plumbing only; no data-path collective)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(per_rank_units: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput of independent replicas: all ranks' units / the slowest rank's time."""
+    return per_rank_units * world / max_seconds
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(PEAK_FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, RuntimeError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def kernel_source_digest(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "bit_kv_cache_24_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name, digest):
+    """DRAM bytes per launch from a committed ncu summary (profiles/<name>.md), or None when the
+    summary is missing or was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"{name}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if line.startswith("- ") and ":" in line:
+            k, v = line[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_digest") != digest:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------------- our arm
+
+class QKVStep:
+    """All buffers of the step, preallocated: no allocation inside the timed region."""
+
+    def __init__(self, device, nsets=3):
+        import bit_kv_cache_24_b200 as nv
+        from bit_kv_cache_24_b200 import synth
+        self.nv = nv
+        self.sets = []
+        for i in range(nsets):
+            d = synth.qkv(seed=1 + 100 * i)
+            self.sets.append({k: v.to(device) for k, v in d.items()})
+        self.A_host = synth.qkv(seed=1)["A"].pin_memory()
+        self.Wq = nv.QTensor(NQKV, HID, nv.SF_MMA, device)
+        self.Aq = nv.QTensor(M_TOK, HID, nv.SF_MMA, device)
+        self.Acq = nv.QTensor(HID, M_TOK, nv.SF_MMA, device)
+        self.amax = torch.empty(1, dtype=torch.float32, device=device)
+        L = nv.lib()
+        self.ws_w = torch.empty(L.nvfp4_quantize_workspace(NQKV, HID), dtype=torch.uint8, device=device)
+        self.ws_a = torch.empty(L.nvfp4_quantize_workspace(M_TOK, HID), dtype=torch.uint8, device=device)
+        self.Y = torch.empty(M_TOK, NQKV, dtype=torch.bfloat16, device=device)
+        self.Y_host = torch.empty(M_TOK, NQKV, dtype=torch.bfloat16).pin_memory()
+        self.cache = nv.KVCache(1, HEADS, HEAD_DIM, SLOTS, M_TOK, device)
+        for s in range(SLOTS):                            # the window: 12 chunks already cached
+            k, v = synth.kv_chunk(0, s)
+            nv.kv_quant_append(self.cache, 0, s, k.to(device), v.to(device))
+        tokens = SLOTS * M_TOK
+        self.Kout = torch.empty(tokens, HEADS, HEAD_DIM, dtype=torch.bfloat16, device=device)
+        self.Vout = torch.empty_like(self.Kout)
+        self.status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.slots = list(range(SLOTS))
+        self.ops = ["w_quantize", "a_amax", "a_quantize_row", "a_quantize_col", "gemm", "kv_append", "kv_dequant"]
+        self.launches_per_step = 2 + 2 + 1 + 1 + 1 + 2 + 1
+
+    def step(self, i, events=None, A=None):
+        nv = self.nv
+        s = self.sets[i % len(self.sets)]
+        A = s["A"] if A is None else A
+        ev = events
+
+        def mark(j):
+            if ev is not None:
+                ev[j].record()
+        mark(0)
+        nv.nvfp4_quantize(s["W"], nv.ROWWISE, out=self.Wq, ws=self.ws_w, status=self.status)
+        mark(1)
+        nv.nvfp4_amax(A, out=self.amax, ws=self.ws_a, status=self.status)
+        mark(2)
+        nv.nvfp4_quantize(A, nv.ROWWISE, amax_in=self.amax, out=self.Aq, status=self.status)
+        mark(3)
+        nv.nvfp4_quantize(A, nv.COLWISE, amax_in=self.amax, out=self.Acq, status=self.status)
+        mark(4)
+        nv.nvfp4_gemm(self.Aq, self.Wq, bias=s["bias"], out=self.Y, status=self.status)
+        mark(5)
+        nv.kv_quant_append(self.cache, 0, i % SLOTS, self.Y[:, HID:2 * HID], self.Y[:, 2 * HID:],
+                           status=self.status)
+        mark(6)
+        nv.kv_dequant(self.cache, 0, self.slots, k_out=self.Kout, v_out=self.Vout, status=self.status)
+        mark(7)
+
+    # algorithmic work per launch of each op (bytes or FLOPs)
+    @staticmethod
+    def work():
+        mk, nk = M_TOK * HID, NQKV * HID
+        q = 2 + 0.5 + 1 / 16                              # BF16 in, codes + scales out, per element
+        win = SLOTS * M_TOK * HEADS * HEAD_DIM
+        return {
+            "w_quantize": ("hbm", 2 * nk + q * nk),       # amax pass + quantize pass
+            "a_amax": ("hbm", 2 * mk),
+            "a_quantize_row": ("hbm", q * mk),
+            "a_quantize_col": ("hbm", q * mk),
+            "gemm": ("tensor", GEMM_FLOP),
+            "kv_append": ("hbm", 2 * (2 * mk + q * mk)),  # K and V: amax pass + quantize pass
+            "kv_dequant": ("hbm", 2 * win * (0.5 + 1 / 16 + 2)),
+        }
+
+
+def run_ours(args, rank, local_rank, world):
+    dist = init_dist(world, "nccl")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    st = QKVStep(dev)
+    nops = len(st.ops)
+    for i in range(args.warmup):
+        st.step(i)
+    torch.cuda.synchronize()
+    if int(st.status.item()) != 0:
+        raise RuntimeError(f"device status {int(st.status.item())} after warm-up")
+
+    K = args.steps
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nops + 1)] for _ in range(K)]
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(K):
+        st.step(args.warmup + i, events[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    per_op = {op: 0.0 for op in st.ops}
+    for ev in events:
+        for j, op in enumerate(st.ops):
+            per_op[op] += ev[j].elapsed_time(ev[j + 1])
+    status = int(st.status.item())
+    max_s = reduce_max(total_ms / 1e3, dist, dev)
+    value = aggregate(GEMM_FLOP * K / 1e12, world, max_s)
+
+    # end to end through the public API: pinned host A -> device, the step, Y -> pinned host
+    E = args.e2e_steps
+    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    A_dev = torch.empty_like(st.sets[0]["A"])
+    for i in range(3):
+        A_dev.copy_(st.A_host, non_blocking=True)
+        st.step(i, A=A_dev)
+        st.Y_host.copy_(st.Y, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e2e_ev[0].record()
+    for i in range(E):
+        A_dev.copy_(st.A_host, non_blocking=True)
+        st.step(i, A=A_dev)
+        st.Y_host.copy_(st.Y, non_blocking=True)
+    e2e_ev[1].record()
+    torch.cuda.synchronize()
+    e2e_s = reduce_max(e2e_ev[0].elapsed_time(e2e_ev[1]) / 1e3, dist, dev)
+    e2e = {"value": aggregate(GEMM_FLOP * E / 1e12, world, e2e_s), "unit": UNIT,
+           "h2d_bytes_per_step": st.A_host.numel() * 2, "d2h_bytes_per_step": st.Y_host.numel() * 2,
+           "steps": E}
+
+    peaks, peak_src = load_peaks()
+    hbm_peak = float(peaks.get("hbm_gbs", PEAK_FALLBACK["hbm_gbs"]))
+    fp4_peak = float(peaks.get("bf16_tflops_sustained", PEAK_FALLBACK["bf16_tflops_sustained"])) * FP4_OVER_BF16
+    kernels = {}
+    for op, (bound, work) in st.work().items():
+        avg_s = per_op[op] / K / 1e3
+        if bound == "tensor":
+            ach, peak, unit = work / avg_s / 1e12, fp4_peak, "TFLOP/s"
+        else:
+            ach, peak, unit = work / avg_s / 1e9, hbm_peak, "GB/s"
+        kernels[op] = {"bound": bound, "us_per_launch": round(avg_s * 1e6, 2), "achieved": round(ach, 1),
+                       "unit": unit, "peak": round(peak, 1), "frac": round(ach / peak, 4),
+                       "share": round(per_op[op] / sum(per_op.values()), 4)}
+    dominant = max(kernels, key=lambda k: kernels[k]["share"])
+    dk = kernels[dominant]
+    digests = {"gemm": ["gemm.cu", "common.cuh", "launch.h"], "kv_dequant": ["kv_cache.cu", "common.cuh", "launch.h"]}
+    traffic = None
+    if dominant in digests:
+        traffic = profiled_traffic(f"{dominant}_qkv_step", kernel_source_digest(digests[dominant]))
+    roofline = {"kernel": dominant, "bound": dk["bound"], "achieved": dk["achieved"], "peak": dk["peak"],
+                "unit": dk["unit"], "frac": dk["frac"], "traffic": traffic,
+                "peak_source": f"{peak_src} ({'HBM copy' if dk['bound'] == 'hbm' else 'bf16 cuBLAS sustained x 4 (nominal FP4:BF16)'})"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_seconds)
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(max_s * 1e3 / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 acc -> bf16",
+        "data": "synthetic (seeded; QKV-projection shapes of a 5B video DiT, random-init weights)",
+        "config": {"workload": "qkv_chunk_step: A[4680x3072] x W[9216x3072]^T + bias, KV append 4680 tok, "
+                               "KV window 12x4680 tok x 24 heads x 128",
+                   "global_batch": M_TOK * world, "seq_len": SLOTS * M_TOK, "parallelism": f"replicas x{world}",
+                   "l2": "inputs rotate over 3 sets (~300 MB) and each step streams ~1.1 GB (> 126 MB L2)",
+                   "value_def": "GEMM FLOPs per step / device time per step (all 7 ops), summed over replicas"},
+        "gpu_launches": st.launches_per_step * K,
+        "kernels": kernels, "roofline": roofline, "clocks": clk, "e2e": e2e,
+        "device_status": status,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------- oracle arm
+
+def oracle_sample_step(rows, wrows, data, orc, synth):
+    """The step's ops on a row sample: W[wrows] quantize, A[rows] amax/row/col quantize, the fp64
+    GEMM of those rows against W[wrows] (+bias), a `rows`-token KV append and the restore of a
+    12-slot window of `rows` tokens each."""
+    A = data["A"][:rows].contiguous()
+    W = data["W"][:wrows].contiguous()
+    _, qw = orc.quantize(W)
+    st, am = orc.amax(A)
+    _, qa = orc.quantize(A, amax_in=am)
+    _, qc = orc.quantize(A, colwise=True, amax_in=am)
+    orc.gemm_rows(qa, qw, bias=data["bias"][:wrows].contiguous(), threads=os.cpu_count())
+    kv = orc.KVCacheModel(1, HEADS, HEAD_DIM, SLOTS, rows)
+    for s in range(SLOTS):
+        kv.append(0, s, data["K"][s], data["V"][s])
+    kv.dequant(0, list(range(SLOTS)))
+    return 2.0 * rows * wrows * HID
+
+
+def oracle_data(rows):
+    from bit_kv_cache_24_b200 import synth
+    d = synth.qkv()
+    k, v = synth.kv_chunk(0, 0)
+    d["K"] = [k[:rows].contiguous()] * SLOTS
+    d["V"] = [v[:rows].contiguous()] * SLOTS
+    return d
+
+
+def cpu_baseline(seconds, rows=16, wrows=256):
+    from oracle import oracle as orc
+    from bit_kv_cache_24_b200 import synth
+    orc.build()
+    data = oracle_data(rows)
+    flop, t0, n = 0.0, time.perf_counter(), 0
+    while True:
+        flop += oracle_sample_step(rows, wrows, data, orc, synth)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": flop / dt / 1e12, "unit": UNIT, "cores": min(os.cpu_count(), rows), "kind": "oracle",
+            "sample": f"{n} oracle steps on A rows [:{rows}] x W rows [:{wrows}] (of 4680 x 9216), "
+                      f"{rows}-token KV append, 12x{rows}-token KV restore; {dt:.1f} s; the fp64 GEMM "
+                      f"runs on {min(os.cpu_count(), rows)} threads, the codecs on one"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from oracle import oracle as orc
+    from bit_kv_cache_24_b200 import synth
+    orc.build()
+    total = args.steps + args.warmup
+    budget = min(1.0, 150.0 / max(1, total))              # seconds per sample step
+    rows = max(1, min(16, int(budget / 0.025)))
+    wrows = 16 * rows
+    data = oracle_data(rows)
+    for _ in range(args.warmup):
+        oracle_sample_step(rows, wrows, data, orc, synth)
+    flop, t0 = 0.0, time.perf_counter()
+    for _ in range(args.steps):
+        flop += oracle_sample_step(rows, wrows, data, orc, synth)
+    dt = time.perf_counter() - t0
+    value = flop / dt / 1e12
+    sample = (f"each step: A rows [:{rows}] x W rows [:{wrows}] (of 4680 x 9216), {rows}-token KV append, "
+              f"12x{rows}-token KV restore")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
+            "data": "synthetic (seeded; same generator as the GPU arm)",
+            "config": {"workload": "qkv_chunk_step (CPU oracle on a row sample)", "global_batch": rows,
+                       "seq_len": SLOTS * rows, "parallelism": "cpu"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(os.cpu_count(), rows), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_ours(args, rank, local_rank, world)
+
+
+if __name__ == "__main__":
+    main()

@@ -73,32 +73,49 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(128 >> 4) << 32) | (1ull << 46);
 }
 
+// The issue helpers below are executed by all 32 lanes of a converged warp with warp-uniform
+// operands; elect.sync picks the one lane that issues.  Issuing from a divergent lane-0 branch
+// instead makes the compiler move every operand into uniform registers lane by lane, which costs
+// ~100 cycles per instruction and starves the tensor core.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int x, int y, uint32_t bar) {
-    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n\t}"
                  :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}"
                  :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void arrive_expect_tx_elect(uint32_t bar, uint32_t bytes) {
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}"
+                 :: "r"(bar), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+                 :: "r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t desc) {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(desc) : "memory");
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;\n\t}"
+                 :: "r"(taddr), "l"(desc) : "memory");
 }
 
 __device__ __forceinline__ void tc_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum,
                                        uint32_t sfa, uint32_t sfb) {
-    asm volatile("{\n\t.reg .pred p;\n\t"
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
                  "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
                  :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum), "r"(sfa), "r"(sfb) : "memory");
 }
 
@@ -138,7 +155,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sbase + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + OFF_MISC + 4);
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = __shfl_sync(0xFFFFFFFFu, (int)(threadIdx.x >> 5), 0);   // warp-uniform
+    const int lane = threadIdx.x & 31;
     const int64_t M = args.M, N = args.N, K = args.K;
     const int mt = (int)ceil_div(M, BM), nt = (int)ceil_div(N, BN);
     const int num_tiles = mt * nt;
@@ -167,7 +185,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
+    const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -184,49 +202,50 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     };
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- producer
-        if (lane == 0) {
-            uint32_t stage = 0, phase = 0;
-            uint32_t last_parity[STAGES];
-            bool used[STAGES];
-            for (int i = 0; i < STAGES; ++i) used[i] = false;
-            bool ok = true;
-            for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
-                const int mb = t % mt, nb = t / mt;
-                for (int kt = 0; kt < nkt; ++kt) {
-                    if (!mbar_wait_bounded(bar_empty + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs)) {
-                        give_up();
-                        ok = false;
-                        break;
-                    }
-                    const int nsteps = min(KSTEPS_PER_TILE, ksteps - kt * KSTEPS_PER_TILE);
-                    const uint32_t sf_bytes = (uint32_t)nsteps * 512u;
-                    const bool b_hi = (2 * nb + 1) < b_row_atoms;
-                    const uint32_t bytes = A_STAGE + B_STAGE + sf_bytes * (b_hi ? 3u : 2u);
-                    const uint32_t fb = bar_full + 8 * stage;
-                    mbar_arrive_expect_tx(fb, bytes);
-                    tma_load_2d(base + OFF_A + stage * A_STAGE, &map_a, kt * (BK / 2), mb * BM, fb);
-                    tma_load_2d(base + OFF_B + stage * B_STAGE, &map_b, kt * (BK / 2), nb * BN, fb);
-                    const int64_t k_atom = (int64_t)kt * KSTEPS_PER_TILE;
-                    bulk_load(base + OFF_SFA + stage * SFA_STAGE,
-                              args.a_sf + ((int64_t)mb * ksteps + k_atom) * 512, sf_bytes, fb);
-                    bulk_load(base + OFF_SFB + stage * SFB_STAGE,
-                              args.b_sf + ((int64_t)(2 * nb) * ksteps + k_atom) * 512, sf_bytes, fb);
-                    if (b_hi)
-                        bulk_load(base + OFF_SFB + stage * SFB_STAGE + SFA_STAGE,
-                                  args.b_sf + ((int64_t)(2 * nb + 1) * ksteps + k_atom) * 512, sf_bytes, fb);
-                    used[stage] = true;
-                    last_parity[stage] = phase;
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        // ---------------------------------------------------------------- producer (whole warp,
+        // converged; one elected lane issues)
+        uint32_t stage = 0, phase = 0;
+        uint32_t used = 0, last_parity = 0;               // per-stage bit masks
+        bool ok = true;
+        for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
+            const int mb = t % mt, nb = t / mt;
+            const bool b_hi = (2 * nb + 1) < b_row_atoms;
+            for (int kt = 0; kt < nkt; ++kt) {
+                if (!warp_wait(bar_empty + 8 * stage, phase ^ 1)) {
+                    ok = false;
+                    break;
                 }
+                const int nsteps = min(KSTEPS_PER_TILE, ksteps - kt * KSTEPS_PER_TILE);
+                const uint32_t sf_bytes = (uint32_t)nsteps * 512u;
+                const uint32_t bytes = A_STAGE + B_STAGE + sf_bytes * (b_hi ? 3u : 2u);
+                const uint32_t fb = bar_full + 8 * stage;
+                arrive_expect_tx_elect(fb, bytes);
+                tma_load_2d(base + OFF_A + stage * A_STAGE, &map_a, kt * (BK / 2), mb * BM, fb);
+                tma_load_2d(base + OFF_B + stage * B_STAGE, &map_b, kt * (BK / 2), nb * BN, fb);
+                const int64_t k_atom = (int64_t)kt * KSTEPS_PER_TILE;
+                bulk_load(base + OFF_SFA + stage * SFA_STAGE,
+                          args.a_sf + ((int64_t)mb * ksteps + k_atom) * 512, sf_bytes, fb);
+                bulk_load(base + OFF_SFB + stage * SFB_STAGE,
+                          args.b_sf + ((int64_t)(2 * nb) * ksteps + k_atom) * 512, sf_bytes, fb);
+                if (b_hi)
+                    bulk_load(base + OFF_SFB + stage * SFB_STAGE + SFA_STAGE,
+                              args.b_sf + ((int64_t)(2 * nb + 1) * ksteps + k_atom) * 512, sf_bytes, fb);
+                used |= 1u << stage;
+                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            // every issued copy must land before this CTA's shared memory can be released
+        }
+        // every issued copy must land before this CTA's shared memory can be released
+        if (lane == 0) {
             for (int i = 0; i < STAGES; ++i)
-                if (used[i] && !mbar_wait_bounded(bar_full + 8 * i, last_parity[i], nullptr, kWaitLimitNs))
+                if (((used >> i) & 1u) &&
+                    !mbar_wait_bounded(bar_full + 8 * i, (last_parity >> i) & 1u, nullptr, kWaitLimitNs))
                     give_up();
         }
+        __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
+        // ---------------------------------------------------------------- MMA issuer (whole warp,
+        // converged; one elected lane issues)
         uint32_t stage = 0, phase = 0, acc_phase = 0;
         bool ok = true, issued = false;
         for (int t = blockIdx.x; ok && t < num_tiles; t += gridDim.x) {
@@ -241,37 +260,33 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     break;
                 }
                 tc_fence_after();
-                if (lane == 0) {
-                    const int nsteps = min(KSTEPS_PER_TILE, ksteps - kt * KSTEPS_PER_TILE);
-                    const uint32_t sfa_s = base + OFF_SFA + stage * SFA_STAGE;
-                    const uint32_t sfb_s = base + OFF_SFB + stage * SFB_STAGE;
-                    for (int j = 0; j < nsteps; ++j) {
-                        tc_cp_sf(tmem + SFA_COL + 4 * j, sf_desc(sfa_s + 512 * j));
-                        tc_cp_sf(tmem + SFB_COL + 8 * j, sf_desc(sfb_s + 512 * j));
-                        tc_cp_sf(tmem + SFB_COL + 8 * j + 4, sf_desc(sfb_s + SFA_STAGE + 512 * j));
-                    }
-                    const uint64_t adesc = sw128_desc(base + OFF_A + stage * A_STAGE);
-                    const uint64_t bdesc = sw128_desc(base + OFF_B + stage * B_STAGE);
-                    for (int j = 0; j < nsteps; ++j) {
-                        // a K step is 64 codes = 32 bytes along the swizzled 128-byte row
-                        tc_mma(tmem + ACC_COL, adesc + 2 * j, bdesc + 2 * j, kIdesc, (kt | j) != 0,
-                               tmem + SFA_COL + 4 * j, tmem + SFB_COL + 8 * j);
-                    }
-                    tc_commit(bar_empty + 8 * stage);
-                    issued = true;
+                const int nsteps = min(KSTEPS_PER_TILE, ksteps - kt * KSTEPS_PER_TILE);
+                const uint32_t sfa_s = base + OFF_SFA + stage * SFA_STAGE;
+                const uint32_t sfb_s = base + OFF_SFB + stage * SFB_STAGE;
+                const uint64_t adesc = sw128_desc(base + OFF_A + stage * A_STAGE);
+                const uint64_t bdesc = sw128_desc(base + OFF_B + stage * B_STAGE);
+                for (int j = 0; j < nsteps; ++j) {
+                    tc_cp_sf(tmem + SFA_COL + 4 * j, sf_desc(sfa_s + 512 * j));
+                    tc_cp_sf(tmem + SFB_COL + 8 * j, sf_desc(sfb_s + 512 * j));
+                    tc_cp_sf(tmem + SFB_COL + 8 * j + 4, sf_desc(sfb_s + SFA_STAGE + 512 * j));
                 }
-                __syncwarp();
+                for (int j = 0; j < nsteps; ++j) {
+                    // a K step is 64 codes = 32 bytes along the swizzled 128-byte row
+                    tc_mma(tmem + ACC_COL, adesc + 2 * j, bdesc + 2 * j, kIdesc, (kt | j) != 0,
+                           tmem + SFA_COL + 4 * j, tmem + SFB_COL + 8 * j);
+                }
+                tc_commit(bar_empty + 8 * stage);
+                issued = true;
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
             if (!ok) break;
-            if (lane == 0) tc_commit(bar_tmem_full);
-            __syncwarp();
+            tc_commit(bar_tmem_full);
             acc_phase ^= 1;
         }
-        // wait for every MMA / copy this thread issued before tensor memory is freed
-        if (lane == 0 && issued) {
+        // wait for every MMA / copy issued here before tensor memory is freed
+        if (issued) {
             tc_commit(bar_drain);
-            if (!mbar_wait_bounded(bar_drain, 0, nullptr, kWaitLimitNs)) give_up();
+            if (lane == 0 && !mbar_wait_bounded(bar_drain, 0, nullptr, kWaitLimitNs)) give_up();
         }
         __syncwarp();
     } else {
