@@ -74,6 +74,7 @@ def lib():
             "nvfp4_kv_append_workspace": (_SZ, [_I64, _I32, _I32]),
             "nvfp4_amax": (_I32, [_P, _I64, _I64, _I64, _P, _P, _SZ, _P, _P]),
             "nvfp4_quantize": (_I32, [_P, _I64, _I64, _I64, _I32, _P, ctypes.POINTER(_Tensor), _P, _SZ, _P, _P]),
+            "nvfp4_quantize_noalloc": (_I32, [_P, _I64, _I64, _I64, _I32, ctypes.POINTER(_Tensor), _P, _P]),
             "nvfp4_gemm": (_I32, [ctypes.POINTER(_Tensor), ctypes.POINTER(_Tensor), _P, _P, _P, _I64, _I32, _P, _P]),
             "nvfp4_kv_cache_bytes": (_I64, [_I32, _I32, _I32, _I32, _I32, _I32]),
             "kv_quant_append": (_I32, [ctypes.POINTER(_KVCache), _I32, _I32, _P, _P, _I64, _I64, _P, _SZ, _P, _P]),

@@ -68,6 +68,8 @@ int num_sms() {
     return d ? d->sms : 148;
 }
 
+void record_error(const char *msg) { std::snprintf(g_last_error, sizeof(g_last_error), "%s", msg); }
+
 }  // namespace nvfp4
 
 using namespace nvfp4;

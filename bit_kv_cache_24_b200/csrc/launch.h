@@ -73,4 +73,7 @@ cudaError_t launch_wait_timeout(int32_t *status, int64_t limit_ns, cudaStream_t 
 
 int num_sms();
 
+// Text returned by nvfp4_last_error() on this thread.
+void record_error(const char *msg);
+
 }  // namespace nvfp4

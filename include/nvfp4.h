@@ -177,6 +177,23 @@ NVFP4_API nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, co
                         int32_t nslots, void *k_out_bf16, void *v_out_bf16, int32_t *dev_status,
                         nvfp4_stream stream);
 
+/*
+ * nvfp4_quantize_noalloc -- nvfp4_quantize without a workspace: for callers that cannot
+ * allocate, such as plugin/enqueue hooks of inference engines and embedded host programs that
+ * receive only their input and output buffers and have no allocator or workspace to hand over.
+ * No counterpart in the paper: it is a deployment variant of the quantizer above.
+ * Same arguments, layouts and results as nvfp4_quantize with amax_in = NULL, bit for bit; the
+ * amax partial maxima go to a 4 KB (1024-slot) static device array held by every GPU that loads
+ * the library.  Nothing is allocated.  A launch needing more than 1024 slots (only possible on
+ * GPUs with more than 256 SMs) returns NVFP4_ERR_UNSUPPORTED with a message in
+ * nvfp4_last_error().  All calls share the array: calls whose kernels overlap on the GPU race
+ * and must be ordered on one stream.  The first call on each device looks up the array's device
+ * address; make that first call before any stream capture.
+ */
+NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, int64_t ld, int32_t dir,
+                                              const nvfp4_tensor *out, int32_t *dev_status,
+                                              nvfp4_stream stream);
+
 /* ---- support --------------------------------------------------------------------------------- */
 
 /* Static description of a status code. */
