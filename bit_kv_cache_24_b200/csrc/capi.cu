@@ -277,7 +277,9 @@ nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, const int32_
     if (layer < 0 || layer >= cache->layers || nslots <= 0 || nslots > kMaxDequantSlots) return NVFP4_ERR_INVALID_ARG;
     const int64_t row = (int64_t)cache->heads * cache->head_dim;
     if ((cache->head_dim & 15) || (row & 31)) return NVFP4_ERR_UNSUPPORTED;
-    if (!aligned16(k_out_bf16) || !aligned16(v_out_bf16)) return NVFP4_ERR_UNSUPPORTED;
+    if (!aligned16(k_out_bf16) || !aligned16(v_out_bf16) || !aligned16(cache->codes_k) ||
+        !aligned16(cache->codes_v) || !aligned16(cache->sf_k) || !aligned16(cache->sf_v))
+        return NVFP4_ERR_UNSUPPORTED;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
     static thread_local DequantJob jk, jv;

@@ -5,10 +5,11 @@
 // yourai.pro: "faster FP4 dequantization", in-place quantized cache updates).  The append side
 // is the row-wise quantizer of quantize.cu run on the chunk's K and V in one launch.
 //
-// Design (B200, HBM-bound: 0.5625 B read + 2 B written per element): one warp restores one
-// token row at a time; per step a lane decodes 8 codes (a 4-byte load; the warp reads 128
-// contiguous bytes) with the hardware E2M1 -> f16x2 conversion, scales them in FP32 and writes
-// 16 bytes (the warp writes 512 contiguous bytes).  K and V are the two halves of the grid.
+// Design (B200, HBM-bound: 0.5625 B read + 2 B written per element): a lane restores 32
+// consecutive elements from one 16-byte code load and one 2-byte scale load (the hardware
+// E2M1 -> f16x2 conversion, FP32 scaling, BF16 packing); a warp keeps two 1024-element spans in
+// flight, stages each span's 2 KB of output in shared memory and writes it with one bulk (TMA)
+// store.  K and V are the two halves of the grid.
 // The slot table (which slot's storage feeds which output tokens) is a kernel parameter, so
 // the host builds no device-side state.
 #include "common.cuh"
@@ -20,16 +21,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-
-__device__ __forceinline__ uint32_t ldg_nc_u32(const void *p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ void stg_v4(void *p, uint4 v) {
-    asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
-}
+constexpr int kSpan = 1024;                 // elements of a token row one warp restores per item
+constexpr int kItems = 2;                   // items a warp keeps in flight
 
 // y = BF16(FP32(e2m1 * sf) * g) for 8 codes packed in one word.
 __device__ __forceinline__ uint4 dequant8(uint32_t codes, float sf, float g) {
@@ -45,41 +38,108 @@ __device__ __forceinline__ uint4 dequant8(uint32_t codes, float sf, float g) {
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_nc_u16(const void *p) {
+    unsigned short v;
+    asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void sts_v4(uint32_t saddr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" :: "r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+// Bulk (TMA) store of `bytes` from shared to global memory, issued by one elected lane of a
+// converged warp, tracked in the issuing thread's bulk-async group.
+__device__ __forceinline__ void bulk_store(void *gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t"
+                 "@p cp.async.bulk.commit_group;\n\t}"
+                 :: "l"(gdst), "r"(ssrc), "r"(bytes) : "memory");
+}
+
+// Wait until the bulk stores of this thread have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p cp.async.bulk.wait_group.read 0;\n\t}" ::: "memory");
+}
+
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p cp.async.bulk.wait_group 0;\n\t}" ::: "memory");
+}
+
+// Work item = (token row, 1024-element span): lane l restores elements [32l, 32l+32) of the span
+// from one 16-byte code load and one 2-byte scale load (two 16-blocks), a warp keeps kItems
+// items in flight.  The span's 2 KB of BF16 output is staged in shared memory and written with
+// one bulk (TMA) store, so global writes are whole contiguous lines.
 __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const __grid_constant__ DequantJob jk,
                                                               const __grid_constant__ DequantJob jv) {
+    __shared__ __align__(128) uint8_t stage[kWarps][kItems][kSpan * 2];
     const DequantJob &j = blockIdx.y == 0 ? jk : jv;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t row_bytes = j.row_elems >> 1, row_sf = j.row_elems >> 4, chunks = j.row_elems >> 3;
-    for (int64_t r = (int64_t)blockIdx.x * kWarps + warp; r < j.total_tokens; r += (int64_t)gridDim.x * kWarps) {
-        // slot holding output token r: last slot with tok_begin <= r (warp-uniform search)
-        int lo = 0, hi = j.nslots - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (j.slot[mid].tok_begin <= r) lo = mid; else hi = mid - 1;
-        }
-        const DequantSlot &s = j.slot[lo];
-        const int64_t t = r - s.tok_begin;
-        const uint8_t *codes = s.codes + t * row_bytes;
-        const uint8_t *sf = s.sf + t * row_sf;
-        const float g = *s.g;
-        uint16_t *out = j.out + r * j.row_elems;
-        int64_t c = lane;
-        for (; c + 96 < chunks; c += 128) {
-            uint32_t w[4];
-            float f[4];
+    const int lane = threadIdx.x & 31;
+    const int warp = __shfl_sync(0xFFFFFFFFu, (int)(threadIdx.x >> 5), 0);
+    const int64_t row_bytes = j.row_elems >> 1, row_sf = j.row_elems >> 4;
+    const int64_t spans = (j.row_elems + kSpan - 1) / kSpan;
+    const int64_t items = j.total_tokens * spans;
+    const int64_t stride = (int64_t)gridDim.x * kWarps * kItems;
+    for (int64_t it0 = ((int64_t)blockIdx.x * kWarps + warp) * kItems; it0 < items; it0 += stride) {
+        uint4 cw[kItems];
+        uint32_t sfw[kItems];
+        float gv[kItems];
+        int64_t r[kItems], e[kItems];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                w[u] = ldg_nc_u32(codes + 4 * (c + 32 * u));
-                f[u] = e4m3_to_f32(sf[(c + 32 * u) >> 1]);
+        for (int u = 0; u < kItems; ++u) {
+            const int64_t it = it0 + u;
+            r[u] = it / spans;
+            e[u] = (it - r[u] * spans) * kSpan;
+            cw[u] = make_uint4(0, 0, 0, 0);
+            sfw[u] = 0;
+            gv[u] = 0.0f;
+            if (it < items) {
+                // slot holding output token r: last slot with tok_begin <= r (warp-uniform search)
+                int lo = 0, hi = j.nslots - 1;
+                while (lo < hi) {
+                    const int mid = (lo + hi + 1) >> 1;
+                    if (j.slot[mid].tok_begin <= r[u]) lo = mid; else hi = mid - 1;
+                }
+                const DequantSlot &sl = j.slot[lo];
+                const int64_t t = r[u] - sl.tok_begin;
+                const int64_t el = e[u] + lane * 32;
+                gv[u] = *sl.g;
+                if (el < j.row_elems) {
+                    cw[u] = ldg_nc_v4(sl.codes + t * row_bytes + (el >> 1));
+                    sfw[u] = ldg_nc_u16(sl.sf + t * row_sf + (el >> 4));
+                }
             }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) stg_v4(out + 8 * (c + 32 * u), dequant8(w[u], f[u], g));
         }
-        for (; c < chunks; c += 32) {
-            const uint32_t w = ldg_nc_u32(codes + 4 * c);
-            stg_v4(out + 8 * c, dequant8(w, e4m3_to_f32(sf[c >> 1]), g));
+        bulk_wait_read();                                 // the previous iteration's stores left smem
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kItems; ++u) {
+            const uint32_t sb = smem_addr(&stage[warp][u][lane * 64]);
+            const float s0 = e4m3_to_f32(sfw[u] & 0xFFu), s1 = e4m3_to_f32(sfw[u] >> 8);
+            sts_v4(sb, dequant8(cw[u].x, s0, gv[u]));
+            sts_v4(sb + 16, dequant8(cw[u].y, s0, gv[u]));
+            sts_v4(sb + 32, dequant8(cw[u].z, s1, gv[u]));
+            sts_v4(sb + 48, dequant8(cw[u].w, s1, gv[u]));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // smem writes -> async proxy
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < kItems; ++u) {
+            if (it0 + u >= items) break;
+            const int64_t n = j.row_elems - e[u] < kSpan ? j.row_elems - e[u] : kSpan;
+            bulk_store(j.out + r[u] * j.row_elems + e[u], smem_addr(&stage[warp][u][0]), (uint32_t)(n * 2));
         }
     }
+    bulk_wait_all();                                      // stores done before shared memory goes away
 }
 
 }  // namespace
@@ -88,7 +148,8 @@ cudaError_t launch_kv_dequant(const DequantJob *k, const DequantJob *v, int32_t 
     (void)status;
     const int64_t tokens = k->total_tokens;
     if (tokens <= 0) return cudaSuccess;
-    int64_t blocks = ceil_div(tokens, kWarps);
+    const int64_t items = tokens * ((k->row_elems + kSpan - 1) / kSpan);
+    int64_t blocks = ceil_div(items, (int64_t)kWarps * kItems);
     const int64_t cap = 8 * (int64_t)num_sms();
     if (blocks > cap) blocks = cap;
     kv_dequant_kernel<<<dim3((unsigned)blocks, 2), kThreads, 0, s>>>(*k, *v);

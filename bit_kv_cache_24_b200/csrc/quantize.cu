@@ -20,6 +20,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+constexpr int kAmaxUnroll = 8;     // 16-byte loads in flight per lane in the amax pass
+constexpr int kRowGroup = 4;       // 256-element segments a warp quantizes per iteration
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
     uint4 v;
@@ -81,12 +83,15 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const __grid_con
     for (int64_t row = (int64_t)blockIdx.x * kWarps + warp; row < j.rows; row += (int64_t)gridDim.x * kWarps) {
         const uint16_t *xr = j.x + row * j.ld;
         int64_t c = lane;
-        for (; c + 96 < cpr; c += 128) {                  // 4 loads in flight per lane
-            uint4 v0 = ldg_nc_v4(xr + 8 * c), v1 = ldg_nc_v4(xr + 8 * (c + 32));
-            uint4 v2 = ldg_nc_v4(xr + 8 * (c + 64)), v3 = ldg_nc_v4(xr + 8 * (c + 96));
-            uint32_t w0[4] = {v0.x, v0.y, v0.z, v0.w}, w1[4] = {v1.x, v1.y, v1.z, v1.w};
-            uint32_t w2[4] = {v2.x, v2.y, v2.z, v2.w}, w3[4] = {v3.x, v3.y, v3.z, v3.w};
-            m = max(m, max(max(absmax_bits8(w0), absmax_bits8(w1)), max(absmax_bits8(w2), absmax_bits8(w3))));
+        for (; c + 32 * (kAmaxUnroll - 1) < cpr; c += 32 * kAmaxUnroll) {   // kAmaxUnroll loads in flight
+            uint4 v[kAmaxUnroll];
+#pragma unroll
+            for (int u = 0; u < kAmaxUnroll; ++u) v[u] = ldg_nc_v4(xr + 8 * (c + 32 * u));
+#pragma unroll
+            for (int u = 0; u < kAmaxUnroll; ++u) {
+                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                m = max(m, absmax_bits8(w));
+            }
         }
         for (; c < cpr; c += 32) {
             uint4 v = ldg_nc_v4(xr + 8 * c);
@@ -139,26 +144,37 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_co
     const int64_t code_cols = 32 * ceil_div(j.cols, 32);
     const int64_t rows_total = mma ? 128 * ceil_div(j.rows, 128) : j.rows;
     const int64_t nseg = ceil_div(mma ? 16 * nb_pad : code_cols, 256);
-    const int64_t items = rows_total * nseg;
+    const int64_t ngrp = ceil_div(nseg, kRowGroup);
+    const int64_t items = rows_total * ngrp;
 
     for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < items; it += (int64_t)gridDim.x * kWarps) {
-        const int64_t row = it / nseg;
-        const int64_t e = (it - row * nseg) * 256 + lane * 8;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (row < j.rows && e < j.cols) v = ldg_nc_v4(j.x + row * j.ld + e);
-        uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t bm = absmax_bits8(w);
-        bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
-        const BlockScale s = block_scale(__uint_as_float(bm << 16), g, den);
-        const uint32_t codes = (s.r == 0.0f) ? 0u : encode8(w, s);
-        if (row < j.rows && e < code_cols)
-            *reinterpret_cast<uint32_t *>(j.codes + row * j.pitch + (e >> 1)) = codes;
-        if ((lane & 1) == 0) {
-            const int64_t blk = e >> 4;
-            if (!mma) {
-                if (row < j.rows && blk < nb) j.sf[row * nb + blk] = (uint8_t)s.sf;
-            } else if (blk < nb_pad) {
-                j.sf[sf_mma_offset(row, blk, atoms)] = (uint8_t)s.sf;
+        const int64_t row = it / ngrp;
+        const int64_t e0 = (it - row * ngrp) * (256 * kRowGroup) + lane * 8;
+        uint4 v[kRowGroup];
+#pragma unroll
+        for (int u = 0; u < kRowGroup; ++u) {           // all loads of the group first
+            const int64_t e = e0 + 256 * u;
+            v[u] = make_uint4(0, 0, 0, 0);
+            if (row < j.rows && e < j.cols) v[u] = ldg_nc_v4(j.x + row * j.ld + e);
+        }
+#pragma unroll
+        for (int u = 0; u < kRowGroup; ++u) {
+            const int64_t e = e0 + 256 * u;
+            if (e >= nseg * 256) break;                 // past the last segment (warp-uniform)
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t bm = absmax_bits8(w);
+            bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
+            const BlockScale sc = block_scale(__uint_as_float(bm << 16), g, den);
+            const uint32_t codes = (sc.r == 0.0f) ? 0u : encode8(w, sc);
+            if (row < j.rows && e < code_cols)
+                *reinterpret_cast<uint32_t *>(j.codes + row * j.pitch + (e >> 1)) = codes;
+            if ((lane & 1) == 0) {
+                const int64_t blk = e >> 4;
+                if (!mma) {
+                    if (row < j.rows && blk < nb) j.sf[row * nb + blk] = (uint8_t)sc.sf;
+                } else if (blk < nb_pad) {
+                    j.sf[sf_mma_offset(row, blk, atoms)] = (uint8_t)sc.sf;
+                }
             }
         }
     }
@@ -271,7 +287,7 @@ __global__ void wait_timeout_kernel(int32_t *status, int64_t limit_ns) {
 
 int amax_blocks(int64_t rows) {
     int64_t b = ceil_div(rows, kWarps);
-    const int64_t cap = 4 * (int64_t)num_sms();
+    const int64_t cap = 6 * (int64_t)num_sms();          // 6 x 256 threads per SM
     if (b > cap) b = cap;
     if (b > kMaxPartials) b = kMaxPartials;
     return (int)(b < 1 ? 1 : b);
@@ -289,7 +305,7 @@ cudaError_t launch_quantize_rows(const RowJobs &jobs, int32_t *status, cudaStrea
     for (int i = 0; i < jobs.njobs; ++i) {
         const RowJob &j = jobs.job[i];
         const int64_t rows = j.sf_layout ? 128 * ceil_div(j.rows, 128) : j.rows;
-        const int64_t it = rows * ceil_div(64 * ceil_div(j.cols, 64), 256);
+        const int64_t it = rows * ceil_div(ceil_div(64 * ceil_div(j.cols, 64), 256), kRowGroup);
         if (it > items) items = it;
     }
     int64_t blocks = ceil_div(items, kWarps);
