@@ -396,6 +396,7 @@ bool make_code_map(CUtensorMap *map, const void *ptr, int64_t rows, int64_t pitc
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs &args, cudaStream_t s) {
+    if (args.M > BM) return launch_gemm_2sm(args, s);     // CTA pairs once M spans two row blocks
     static bool attr_set[64] = {false};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

@@ -67,6 +67,8 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm(const GemmArgs &args, cudaStream_t s);
+// CTA-pair (cta_group::2) variant for M > 128; launch_gemm dispatches to it.
+cudaError_t launch_gemm_2sm(const GemmArgs &args, cudaStream_t s);
 
 cudaError_t launch_encode_elements(const float *in, int64_t n, uint8_t *e2m1_out, uint8_t *e4m3_out, cudaStream_t s);
 cudaError_t launch_wait_timeout(int32_t *status, int64_t limit_ns, cudaStream_t s);
