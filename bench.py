@@ -326,7 +326,8 @@ def run_ours(args, rank, local_rank, world):
                        "share": round(per_op[op] / sum(per_op.values()), 4)}
     dominant = max(kernels, key=lambda k: kernels[k]["share"])
     dk = kernels[dominant]
-    digests = {"gemm": ["gemm.cu", "common.cuh", "launch.h"], "kv_dequant": ["kv_cache.cu", "common.cuh", "launch.h"]}
+    digests = {"gemm": ["gemm.cu", "gemm2sm.cu", "common.cuh", "launch.h"],
+               "kv_dequant": ["kv_cache.cu", "common.cuh", "launch.h"]}
     traffic = None
     if dominant in digests:
         traffic = profiled_traffic(f"{dominant}_qkv_step", kernel_source_digest(digests[dominant]))

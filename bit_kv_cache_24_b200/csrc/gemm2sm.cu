@@ -159,28 +159,6 @@ __device__ __forceinline__ void stg_v4(void *p, uint4 v) {
     asm volatile("st.global.v4.u32 [%0], {%1, %2, %3, %4};" :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// Bounded wait with cluster-scope acquire (for barriers that remote CTAs arrive on).
-__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const volatile int *abort,
-                                                  uint64_t limit_ns) {
-    auto try_once = [&]() {
-        uint32_t done;
-        asm volatile("{\n\t.reg .pred p;\n\t"
-                     "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-                     "selp.u32 %0, 1, 0, p;\n\t}"
-                     : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-        return done != 0;
-    };
-    if (try_once()) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (try_once()) return true;
-        if ((it & 255u) == 0) {
-            if (abort && *abort) return false;
-            if (globaltimer_ns() - t0 > limit_ns) return false;
-        }
-    }
-}
-
 struct Maps {
     CUtensorMap a, b, sfa, sfb;
 };
@@ -215,7 +193,7 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
             mbar_init(bar_sf + 8 * i, 1);
         }
         mbar_init(bar_tmem_full, 1);
-        mbar_init(bar_tmem_empty, 2 * EPI_WARPS * 32);
+        mbar_init(bar_tmem_empty, 2 * EPI_WARPS);          // one arrival per epilogue warp of the pair
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -311,7 +289,7 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
         for (int t = cluster; ok && t < num_tiles; t += nclusters) {
             bool got = true;
             if (lane == 0) {
-                got = mbar_wait_cluster(bar_tmem_empty, acc_phase ^ 1, abort_flag, kWaitLimitNs);
+                got = mbar_wait_bounded(bar_tmem_empty, acc_phase ^ 1, abort_flag, kWaitLimitNs);
                 if (!got) give_up();
             }
             if (!__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0)) break;
@@ -363,7 +341,9 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
             for (int c = 0; c < 4; ++c) tc_ld32_nowait(trow + c * 32, r[c]);
             asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
             tc_fence_before();
-            asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(lead_tmem_empty) : "memory");
+            __syncwarp();
+            if (lane == 0)
+                asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" :: "r"(lead_tmem_empty) : "memory");
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int64_t n0 = (int64_t)nb * BN + half * 128 + c * 32;
