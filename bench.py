@@ -3,9 +3,9 @@
 projection of a 5B-class video DiT layer with every NVFP4 operation of the path:
 
   a4  weight quantize        W [9216 x 3072] BF16 -> NVFP4 (re-quantized each step, as in training)
-  a1  activation amax        A [4680 x 3072] (3 latent frames x 30 x 52 patches)
-  a2  row-wise quantize      A -> GEMM operand (amax reused)
-  a3  column-wise quantize   A -> token-dim blocks (the wgrad operand; amax reused)
+  a1-a3 activation quantize  A [4680 x 3072] (3 latent frames x 30 x 52 patches): amax, row-wise
+                             (GEMM operand) and column-wise (token-dim blocks, the wgrad operand)
+                             from one read of A
   a5+a6 NVFP4 GEMM + bias    Y [4680 x 9216] = gA*gB * A.W^T + bias, BF16
   a7  KV append              K = Y[:, 3072:6144], V = Y[:, 6144:] (strided) -> cache slot (in place)
   a8  KV restore             the 12-slot window (56160 tokens, 24 heads x 128) -> BF16 K and V
@@ -189,7 +189,6 @@ class QKVStep:
         self.Wq = nv.QTensor(NQKV, HID, nv.SF_MMA, device)
         self.Aq = nv.QTensor(M_TOK, HID, nv.SF_MMA, device)
         self.Acq = nv.QTensor(HID, M_TOK, nv.SF_MMA, device)
-        self.amax = torch.empty(1, dtype=torch.float32, device=device)
         L = nv.lib()
         self.ws_w = torch.empty(L.nvfp4_quantize_workspace(NQKV, HID), dtype=torch.uint8, device=device)
         self.ws_a = torch.empty(L.nvfp4_quantize_workspace(M_TOK, HID), dtype=torch.uint8, device=device)
@@ -204,8 +203,10 @@ class QKVStep:
         self.Vout = torch.empty_like(self.Kout)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
         self.slots = list(range(SLOTS))
-        self.ops = ["w_quantize", "a_amax", "a_quantize_row", "a_quantize_col", "gemm", "kv_append", "kv_dequant"]
-        self.launches_per_step = 2 + 2 + 1 + 1 + 1 + 2 + 1
+        self.ops = ["w_quantize", "a_quantize_rowcol", "gemm", "kv_append", "kv_dequant"]
+        # kernels per step: W amax + scale record + row pass; A amax + record + row + column pass;
+        # GEMM; K/V amax + record + row pass (both tensors per launch); dequant
+        self.launches_per_step = 3 + 4 + 1 + 3 + 1
 
     def step(self, i, events=None, A=None):
         nv = self.nv
@@ -219,19 +220,15 @@ class QKVStep:
         mark(0)
         nv.nvfp4_quantize(s["W"], nv.ROWWISE, out=self.Wq, ws=self.ws_w, status=self.status)
         mark(1)
-        nv.nvfp4_amax(A, out=self.amax, ws=self.ws_a, status=self.status)
+        nv.nvfp4_quantize(A, nv.ROWCOL, out=(self.Aq, self.Acq), ws=self.ws_a, status=self.status)
         mark(2)
-        nv.nvfp4_quantize(A, nv.ROWWISE, amax_in=self.amax, out=self.Aq, status=self.status)
-        mark(3)
-        nv.nvfp4_quantize(A, nv.COLWISE, amax_in=self.amax, out=self.Acq, status=self.status)
-        mark(4)
         nv.nvfp4_gemm(self.Aq, self.Wq, bias=s["bias"], out=self.Y, status=self.status)
-        mark(5)
+        mark(3)
         nv.kv_quant_append(self.cache, 0, i % SLOTS, self.Y[:, HID:2 * HID], self.Y[:, 2 * HID:],
                            status=self.status)
-        mark(6)
+        mark(4)
         nv.kv_dequant(self.cache, 0, self.slots, k_out=self.Kout, v_out=self.Vout, status=self.status)
-        mark(7)
+        mark(5)
 
     # algorithmic work per launch of each op (bytes or FLOPs)
     @staticmethod
@@ -240,12 +237,12 @@ class QKVStep:
         q = 2 + 0.5 + 1 / 16                              # BF16 in, codes + scales out, per element
         win = SLOTS * M_TOK * HEADS * HEAD_DIM
         return {
-            "w_quantize": ("hbm", 2 * nk + q * nk),       # amax pass + quantize pass
-            "a_amax": ("hbm", 2 * mk),
-            "a_quantize_row": ("hbm", q * mk),
-            "a_quantize_col": ("hbm", q * mk),
+            # bytes that must cross HBM at least once per op: BF16 in (read once), codes + scales
+            # out; the second read of the two-pass quantizers is not counted
+            "w_quantize": ("hbm", q * nk),
+            "a_quantize_rowcol": ("hbm", (2 + 2 * (0.5 + 1 / 16)) * mk),   # both layouts from one read
             "gemm": ("tensor", GEMM_FLOP),
-            "kv_append": ("hbm", 2 * (2 * mk + q * mk)),  # K and V: amax pass + quantize pass
+            "kv_append": ("hbm", 2 * q * mk),                # K and V
             "kv_dequant": ("hbm", 2 * win * (0.5 + 1 / 16 + 2)),
         }
 

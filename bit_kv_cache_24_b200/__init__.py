@@ -25,7 +25,7 @@ HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
 NVFP4_OK, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_UNSUPPORTED = 0, 1, 2
 NVFP4_ERR_NONFINITE, NVFP4_ERR_TIMEOUT, NVFP4_ERR_CUDA = 3, 4, 5
-ROWWISE, COLWISE = 0, 1
+ROWWISE, COLWISE, ROWCOL = 0, 1, 2
 SF_LINEAR, SF_MMA = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 
@@ -155,16 +155,23 @@ def nvfp4_amax(x, out=None, ws=None, status=None, stream=None):
 
 
 def nvfp4_quantize(x, dir=ROWWISE, amax_in=None, out=None, sf_layout=SF_MMA, ws=None, status=None, stream=None):
-    """BF16 [M, K] -> NVFP4.  Row-wise: out is [M, K]; column-wise: out is [K, M] (blocks along M)."""
+    """BF16 [M, K] -> NVFP4.  Row-wise: out is [M, K]; column-wise: out is [K, M] (blocks along M);
+    ROWCOL: both from one read, out = (row-wise [M, K], column-wise [K, M])."""
     x = _bf16_2d(x, "x")
     L = lib()
     M, K = x.shape
     if out is None:
-        out = QTensor(M, K, sf_layout, x.device) if dir == ROWWISE else QTensor(K, M, sf_layout, x.device)
-    if ws is None and amax_in is None:
+        if dir == ROWWISE:
+            out = QTensor(M, K, sf_layout, x.device)
+        elif dir == COLWISE:
+            out = QTensor(K, M, sf_layout, x.device)
+        else:
+            out = (QTensor(M, K, sf_layout, x.device), QTensor(K, M, sf_layout, x.device))
+    if ws is None:
         ws = _ws(L.nvfp4_quantize_workspace(M, K), x.device)
-    st = out.struct()
-    _check("nvfp4_quantize", L.nvfp4_quantize(_ptr(x), M, K, x.stride(0), dir, _ptr(amax_in), ctypes.byref(st),
+    outs = out if isinstance(out, tuple) else (out,)
+    st = (_Tensor * len(outs))(*[o.struct() for o in outs])
+    _check("nvfp4_quantize", L.nvfp4_quantize(_ptr(x), M, K, x.stride(0), dir, _ptr(amax_in), st,
                                               _ptr(ws), 0 if ws is None else ws.numel(), _ptr(status),
                                               _stream(stream)))
     return out

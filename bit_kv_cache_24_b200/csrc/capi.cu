@@ -61,6 +61,16 @@ int64_t sf_bytes(int64_t rows, int64_t cols, int32_t layout) {
     return -1;
 }
 
+// The quantizers index the units of one tensor, padding included, with 32-bit integers.
+bool too_large(int64_t rows, int64_t cols) {
+    return (uint64_t)(rows + 128) * (uint64_t)(cols + 128) >= (1ull << 35);
+}
+
+bool tensor_ok(const nvfp4_tensor *t, int64_t rows, int64_t cols) {
+    return t && t->codes && t->sf && t->g && t->rows == rows && t->cols == cols &&
+           (t->sf_layout == NVFP4_SF_LINEAR || t->sf_layout == NVFP4_SF_MMA);
+}
+
 }  // namespace
 
 int num_sms() {
@@ -99,21 +109,21 @@ int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols, int32_t layout) { return sf_b
 size_t nvfp4_quantize_workspace(int64_t rows, int64_t cols) {
     (void)rows;
     (void)cols;
-    return (size_t)kMaxPartials * sizeof(uint32_t);
+    return kTensorScratchBytes;
 }
 
 size_t nvfp4_kv_append_workspace(int64_t ntok, int32_t heads, int32_t head_dim) {
     (void)ntok;
     (void)heads;
     (void)head_dim;
-    return 2 * (size_t)kMaxPartials * sizeof(uint32_t);
+    return 2 * kTensorScratchBytes;
 }
 
 nvfp4_status nvfp4_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ld, float *amax_out, void *ws,
                         size_t ws_bytes, int32_t *dev_status, nvfp4_stream stream) {
     if (!x_bf16 || !amax_out || !ws || M < 0 || K < 0 || ld < K) return NVFP4_ERR_INVALID_ARG;
     if (ws_bytes < nvfp4_quantize_workspace(M, K)) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(x_bf16) || !aligned16(ws) || (ld & 7) || (K & 7)) return NVFP4_ERR_UNSUPPORTED;
+    if (!aligned16(x_bf16) || !aligned16(ws) || (ld & 7) || (K & 7) || too_large(M, K)) return NVFP4_ERR_UNSUPPORTED;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
     RowJobs jobs{};
@@ -131,20 +141,24 @@ nvfp4_status nvfp4_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ld, fl
 nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld, int32_t dir,
                             const float *amax_in, const nvfp4_tensor *out, void *ws, size_t ws_bytes,
                             int32_t *dev_status, nvfp4_stream stream) {
-    if (!x_bf16 || !out || !out->codes || !out->sf || !out->g || M <= 0 || K <= 0 || ld < K)
-        return NVFP4_ERR_INVALID_ARG;
-    if (dir != NVFP4_ROWWISE && dir != NVFP4_COLWISE) return NVFP4_ERR_INVALID_ARG;
-    if (out->sf_layout != NVFP4_SF_LINEAR && out->sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_INVALID_ARG;
-    const int64_t orows = dir == NVFP4_ROWWISE ? M : K, ocols = dir == NVFP4_ROWWISE ? K : M;
-    if (out->rows != orows || out->cols != ocols) return NVFP4_ERR_INVALID_ARG;
-    if (!amax_in && (!ws || ws_bytes < nvfp4_quantize_workspace(M, K))) return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(x_bf16) || (ld & 7) || (K & 7)) return NVFP4_ERR_UNSUPPORTED;
-    if (dir == NVFP4_ROWWISE && (K & 15)) return NVFP4_ERR_UNSUPPORTED;
-    if (!aligned16(out->codes) || (ws && !aligned16(ws))) return NVFP4_ERR_UNSUPPORTED;
+    if (!x_bf16 || !out || M <= 0 || K <= 0 || ld < K) return NVFP4_ERR_INVALID_ARG;
+    if (dir != NVFP4_ROWWISE && dir != NVFP4_COLWISE && dir != NVFP4_ROWCOL) return NVFP4_ERR_INVALID_ARG;
+    const nvfp4_tensor *row_out = dir != NVFP4_COLWISE ? &out[0] : nullptr;
+    const nvfp4_tensor *col_out = dir == NVFP4_COLWISE ? &out[0] : (dir == NVFP4_ROWCOL ? &out[1] : nullptr);
+    if (row_out && !tensor_ok(row_out, M, K)) return NVFP4_ERR_INVALID_ARG;
+    if (col_out && !tensor_ok(col_out, K, M)) return NVFP4_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < nvfp4_quantize_workspace(M, K)) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16) || (ld & 7) || (K & 7) || too_large(M, K)) return NVFP4_ERR_UNSUPPORTED;
+    if (row_out && (K & 15)) return NVFP4_ERR_UNSUPPORTED;
+    if ((row_out && !aligned16(row_out->codes)) || (col_out && !aligned16(col_out->codes)) || !aligned16(ws))
+        return NVFP4_ERR_UNSUPPORTED;
     nvfp4_status st = check_device();
     if (st != NVFP4_OK) return st;
-
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *scratch = static_cast<uint8_t *>(ws);
+    ScaleRecord *rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
+
+    // amax pass (unless amax_in), the scale record, then one pass per requested layout
     RowJobs jobs{};
     jobs.njobs = 1;
     jobs.npartial = amax_blocks(M);
@@ -153,22 +167,33 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
     j.rows = M;
     j.cols = K;
     j.ld = ld;
-    j.codes = out->codes;
-    j.pitch = codes_pitch(ocols);
-    j.sf = out->sf;
-    j.sf_layout = out->sf_layout;
-    j.g_out = out->g;
-    j.amax_in = amax_in;
-    j.partial = static_cast<uint32_t *>(ws);
+    j.partial = reinterpret_cast<uint32_t *>(scratch);
+    j.rec = rec;
+    RecJobs rj{};
+    rj.njobs = 1;
+    rj.npartial = jobs.npartial;
+    rj.job[0].partial = j.partial;
+    rj.job[0].amax_in = amax_in;
+    rj.job[0].rec = rec;
+    rj.job[0].g_out[0] = row_out ? row_out->g : nullptr;
+    rj.job[0].g_out[1] = col_out ? col_out->g : nullptr;
     cudaError_t e = cudaSuccess;
     if (!amax_in) e = launch_amax(jobs, dev_status, nullptr, s);
-    if (e == cudaSuccess) {
-        if (dir == NVFP4_ROWWISE) {
-            e = launch_quantize_rows(jobs, dev_status, s);
-        } else {
-            RowJob jc = j;
-            e = launch_quantize_cols(jc, jobs.npartial, dev_status, s);
-        }
+    if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+    if (e == cudaSuccess && row_out) {
+        j.codes = row_out->codes;
+        j.pitch = codes_pitch(K);
+        j.sf = row_out->sf;
+        j.sf_layout = row_out->sf_layout;
+        e = launch_quantize_rows(jobs, s);
+    }
+    if (e == cudaSuccess && col_out) {
+        RowJob jc = j;
+        jc.codes = col_out->codes;
+        jc.pitch = codes_pitch(M);
+        jc.sf = col_out->sf;
+        jc.sf_layout = col_out->sf_layout;
+        e = launch_quantize_cols(jc, s);
     }
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_quantize");
 }
@@ -238,7 +263,7 @@ nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int32_t slot,
     const int64_t row = (int64_t)cache->heads * cache->head_dim;
     if (ntok <= 0 || ntok > cache->slot_tokens || ld < row) return NVFP4_ERR_INVALID_ARG;
     if (ws_bytes < nvfp4_kv_append_workspace(ntok, cache->heads, cache->head_dim)) return NVFP4_ERR_INVALID_ARG;
-    if ((cache->head_dim & 15) || (row & 31) || (ld & 7)) return NVFP4_ERR_UNSUPPORTED;
+    if ((cache->head_dim & 15) || (row & 31) || (ld & 7) || too_large(ntok, row)) return NVFP4_ERR_UNSUPPORTED;
     if (!aligned16(k_bf16) || !aligned16(v_bf16) || !aligned16(ws) || !aligned16(cache->codes_k) ||
         !aligned16(cache->codes_v))
         return NVFP4_ERR_UNSUPPORTED;
@@ -246,10 +271,15 @@ nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int32_t slot,
     if (st != NVFP4_OK) return st;
     const int64_t slot_index = (int64_t)layer * cache->slots + slot;
     const int64_t tok0 = slot_index * cache->slot_tokens;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
     RowJobs jobs{};
     jobs.njobs = 2;
     jobs.npartial = amax_blocks(ntok);
+    RecJobs rj{};
+    rj.njobs = 2;
+    rj.npartial = jobs.npartial;
     for (int i = 0; i < 2; ++i) {
+        uint8_t *scratch = static_cast<uint8_t *>(ws) + i * kTensorScratchBytes;
         RowJob &j = jobs.job[i];
         j.x = static_cast<const uint16_t *>(i == 0 ? k_bf16 : v_bf16);
         j.rows = ntok;
@@ -259,13 +289,17 @@ nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int32_t slot,
         j.pitch = row / 2;
         j.sf = (i == 0 ? cache->sf_k : cache->sf_v) + tok0 * (row / 16);
         j.sf_layout = NVFP4_SF_LINEAR;
-        j.g_out = (i == 0 ? cache->g_k : cache->g_v) + slot_index;
-        j.amax_in = nullptr;
-        j.partial = static_cast<uint32_t *>(ws) + i * kMaxPartials;
+        j.partial = reinterpret_cast<uint32_t *>(scratch);
+        j.rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
+        rj.job[i].partial = j.partial;
+        rj.job[i].amax_in = nullptr;
+        rj.job[i].rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
+        rj.job[i].g_out[0] = (i == 0 ? cache->g_k : cache->g_v) + slot_index;
+        rj.job[i].g_out[1] = nullptr;
     }
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = launch_amax(jobs, dev_status, nullptr, s);
-    if (e == cudaSuccess) e = launch_quantize_rows(jobs, dev_status, s);
+    if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+    if (e == cudaSuccess) e = launch_quantize_rows(jobs, s);
     if (e != cudaSuccess) return cuda_fail(e, "kv_quant_append");
     cache->len[slot_index] = (int32_t)ntok;
     return NVFP4_OK;

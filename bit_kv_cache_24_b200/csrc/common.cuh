@@ -24,6 +24,16 @@ constexpr float kE2M1Max = 6.0f;
 constexpr float kE4M3Max = 448.0f;
 constexpr float kGlobalDen = kE2M1Max * kE4M3Max;   // 2688: maps the tensor max to both grid tops
 
+// ---- programmatic dependent launch --------------------------------------------------------------
+//
+// Every kernel of the library is launched with programmatic stream serialization (launch_pdl) and
+// calls griddep_wait() before its first global memory access: that returns once the preceding
+// kernel in the stream has completed and its writes are visible, so only the launch and the
+// prologue overlap the predecessor's tail.  griddep_launch_dependents() (after the wait) lets the
+// next kernel be scheduled early.  Both are no-ops in a launch without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---- status word ------------------------------------------------------------------------------
 
 __device__ __forceinline__ void set_status(int32_t *st, int32_t code) {
@@ -90,21 +100,24 @@ __device__ __forceinline__ float global_scale(float amax) {
 
 // ---- the 16-block quantization step -----------------------------------------------------------
 //
-// Given the block max b (exact BF16 value), g and den = g*6: the scale byte, and r = 1/d
-// (0 when d == 0, meaning every code of the block is +0).
+// A block's scale byte and r = 1/d (0 when d == 0, meaning every code of the block is +0).
 struct BlockScale {
     uint32_t sf;
     float r;
     bool r_inf;   // d so small that 1/d overflows: x*r is then +-inf (or NaN for x == 0)
 };
 
-__device__ __forceinline__ BlockScale block_scale(float b, float g, float den) {
-    BlockScale s;
-    s.sf = (b == 0.0f) ? 0u : e4m3(__fdiv_rn(b, den));
-    const float d = __fmul_rn(e4m3_to_f32(s.sf), g);
-    s.r = (d == 0.0f) ? 0.0f : __frcp_rn(d);
-    s.r_inf = isinf(s.r);
-    return s;
+
+// Two BF16 (one packed word) times r: both products in FP32 (IEEE RN, one paired multiply).
+__device__ __forceinline__ void mul_bf16x2(uint32_t w, float r, float &lo, float &hi) {
+    unsigned long long p;
+    asm("{\n\t.reg .b64 a, b;\n\t"
+        "mov.b64 a, {%1, %2};\n\t"
+        "mov.b64 b, {%3, %3};\n\t"
+        "mul.rn.f32x2 %0, a, b;\n\t}"
+        : "=l"(p) : "r"(w << 16), "r"(w & 0xFFFF0000u), "f"(r));
+    lo = __uint_as_float((uint32_t)p);
+    hi = __uint_as_float((uint32_t)(p >> 32));
 }
 
 // Eight BF16 (as 4 packed words) -> 8 E2M1 codes given the block's reciprocal scale.
@@ -113,10 +126,7 @@ __device__ __forceinline__ BlockScale block_scale(float b, float g, float den) {
 __device__ __forceinline__ uint32_t encode8(const uint32_t w[4], const BlockScale &s) {
     float q[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        q[2 * i] = __fmul_rn(bf16_lo(w[i]), s.r);
-        q[2 * i + 1] = __fmul_rn(bf16_hi(w[i]), s.r);
-    }
+    for (int i = 0; i < 4; ++i) mul_bf16x2(w[i], s.r, q[2 * i], q[2 * i + 1]);
     if (s.r_inf) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -132,6 +142,21 @@ __device__ __forceinline__ uint32_t absmax_bits8(const uint32_t w[4]) {
     uint32_t m = __vmaxu2(w[0] & 0x7FFF7FFFu, w[1] & 0x7FFF7FFFu);
     m = __vmaxu2(m, __vmaxu2(w[2] & 0x7FFF7FFFu, w[3] & 0x7FFF7FFFu));
     return max(m & 0xFFFFu, m >> 16);
+}
+
+// Max of |x| over 16 BF16 in 8 words, as BF16 magnitude bits: paired abs-max (sign bits are
+// masked off at the end), NaN-propagating so that a NaN still compares above 0x7F80.
+__device__ __forceinline__ uint32_t absmax_bits16(const uint32_t w[8]) {
+    uint32_t a, b, c, d;
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(w[0]), "r"(w[1]));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(b) : "r"(w[2]), "r"(w[3]));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(w[4]), "r"(w[5]));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(w[6]), "r"(w[7]));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(a), "r"(b));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(c) : "r"(c), "r"(d));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(a) : "r"(a), "r"(c));
+    a &= 0x7FFF7FFFu;
+    return max(a & 0xFFFFu, a >> 16);
 }
 
 // ---- tensor-core scale layout -----------------------------------------------------------------

@@ -186,6 +186,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
+    griddep_wait();                                       // operands written by earlier kernels
+    griddep_launch_dependents();
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -413,8 +415,7 @@ cudaError_t launch_gemm(const GemmArgs &args, cudaStream_t s) {
     const int64_t tiles = ceil_div(args.M, BM) * ceil_div(args.N, BN);
     int grid = num_sms();
     if (tiles < grid) grid = (int)tiles;
-    nvfp4_gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, s>>>(ma, mb, args);
-    return cudaGetLastError();
+    return launch_pdl(nvfp4_gemm_kernel, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, s, ma, mb, args);
 }
 
 }  // namespace nvfp4

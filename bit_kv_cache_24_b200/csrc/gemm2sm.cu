@@ -213,6 +213,8 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
     cluster_sync();                                       // barriers and tensor memory of both CTAs ready
     tc_fence_after();
     const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
+    griddep_wait();                                       // operands written by earlier kernels
+    griddep_launch_dependents();
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -453,13 +455,15 @@ cudaError_t launch_gemm_2sm(const GemmArgs &args, cudaStream_t s) {
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     cfg.dynamicSmemBytes = SMEM_BYTES;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see griddep_wait
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, nvfp4_gemm_2sm_kernel, maps, args);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

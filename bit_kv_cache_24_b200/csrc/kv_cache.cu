@@ -82,6 +82,8 @@ __device__ __forceinline__ void bulk_wait_all() {
 __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const __grid_constant__ DequantJob jk,
                                                               const __grid_constant__ DequantJob jv) {
     __shared__ __align__(128) uint8_t stage[kWarps][kItems][kSpan * 2];
+    griddep_wait();                                       // the cache written by earlier kernels
+    griddep_launch_dependents();
     const DequantJob &j = blockIdx.y == 0 ? jk : jv;
     const int lane = threadIdx.x & 31;
     const int warp = __shfl_sync(0xFFFFFFFFu, (int)(threadIdx.x >> 5), 0);
@@ -152,8 +154,7 @@ cudaError_t launch_kv_dequant(const DequantJob *k, const DequantJob *v, int32_t 
     int64_t blocks = ceil_div(items, (int64_t)kWarps * kItems);
     const int64_t cap = 8 * (int64_t)num_sms();
     if (blocks > cap) blocks = cap;
-    kv_dequant_kernel<<<dim3((unsigned)blocks, 2), kThreads, 0, s>>>(*k, *v);
-    return cudaGetLastError();
+    return launch_pdl(kv_dequant_kernel, dim3((unsigned)blocks, 2), dim3(kThreads), 0, s, *k, *v);
 }
 
 }  // namespace nvfp4

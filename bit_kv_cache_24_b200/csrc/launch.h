@@ -9,17 +9,31 @@ namespace nvfp4 {
 constexpr int kMaxPartials = 1024;        // per-CTA partial maxima of one amax pass
 constexpr int kMaxJobs = 2;               // tensors quantized by one launch (K and V)
 
-// One tensor to reduce / quantize row-wise.
+// Per-tensor scale record: written once per quantization by the record kernel from the amax,
+// read by every CTA of the quantize passes.
+struct ScaleRecord {
+    uint32_t ok;            // 0: the tensor (or amax_in) was non-finite; the quantize passes skip
+    float g;                // decode scale amax / 2688 (1 when amax == 0)
+    float den;              // g * 6
+    float inv_den;          // RN(1 / den), or 0 when den < 2^-125 (the quotient then divides)
+    float r_tab[128];       // r_tab[sf] = RN(1 / RN(e4m3(sf) * g)), 0 where that product is 0
+};
+
+// Device workspace of one quantized tensor: the amax partials, then its scale record.
+constexpr size_t kRecordOffset = kMaxPartials * sizeof(uint32_t);
+constexpr size_t kTensorScratchBytes = kRecordOffset + 1024;
+static_assert(sizeof(ScaleRecord) <= 1024, "record fits its slot");
+
+// One tensor to reduce / quantize.
 struct RowJob {
     const uint16_t *x;      // BF16 [rows][ld]
     int64_t rows, cols, ld;
-    uint8_t *codes;         // [rows][pitch]
+    uint8_t *codes;         // [rows][pitch] (column-wise: [cols][pitch])
     int64_t pitch;
     uint8_t *sf;
     int32_t sf_layout;      // 0 linear [rows][ceil(cols/16)], 1 tensor-core layout
-    float *g_out;
-    const float *amax_in;   // nullable device pointer
-    uint32_t *partial;      // [kMaxPartials] partial maxima (BF16 magnitude bits)
+    uint32_t *partial;      // [kMaxPartials] partial maxima (BF16 magnitude bits), amax pass
+    const ScaleRecord *rec; // read by the quantize passes
 };
 
 struct RowJobs {
@@ -28,11 +42,42 @@ struct RowJobs {
     int32_t npartial;
 };
 
+// One tensor's scale record: from the partials of its amax pass, or from amax_in when non-null.
+struct RecJob {
+    const uint32_t *partial;
+    const float *amax_in;
+    ScaleRecord *rec;
+    float *g_out[2];        // nullable: receive g (row- and column-wise outputs)
+};
+
+struct RecJobs {
+    RecJob job[kMaxJobs];
+    int32_t njobs;
+    int32_t npartial;
+};
+
 cudaError_t launch_amax(const RowJobs &jobs, int32_t *status, float *amax_out, cudaStream_t s);
-cudaError_t launch_quantize_rows(const RowJobs &jobs, int32_t *status, cudaStream_t s);
+cudaError_t launch_scale_record(const RecJobs &jobs, int32_t *status, cudaStream_t s);
+cudaError_t launch_quantize_rows(const RowJobs &jobs, cudaStream_t s);
 // Column-wise: blocks along the rows of x; output [cols][pitch(rows)].
-cudaError_t launch_quantize_cols(const RowJob &job, int32_t npartial, int32_t *status, cudaStream_t s);
+cudaError_t launch_quantize_cols(const RowJob &job, cudaStream_t s);
 int amax_blocks(int64_t rows);
+
+// Launch with programmatic stream serialization (see griddep_wait in common.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 struct DequantSlot {
     const uint8_t *codes;   // [ntok][row_bytes]

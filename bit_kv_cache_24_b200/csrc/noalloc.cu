@@ -1,20 +1,21 @@
 // noalloc.cu -- nvfp4_quantize_noalloc: the quantizer for callers that cannot allocate.
 //
 // nvfp4_quantize needs a small device workspace for the per-CTA partial maxima of its amax
-// pass.  Some callers have no way to provide one: plugin or enqueue hooks of inference engines
+// pass and the per-tensor scale record.  Some callers have no way to provide one: plugin or enqueue hooks of inference engines
 // and embedded host programs that receive only their input and output buffers and have neither
 // an allocator nor a workspace to hand over (and must not call cudaMalloc on their hot path).
-// This entry point keeps those partials in a file-scope device array instead, so the caller
+// This entry point keeps that scratch in a file-scope device array instead, so the caller
 // passes inputs and outputs only and nothing is allocated.
 //
 // Contract:
-//   - The scratch is kNoAllocPartials (1024) 32-bit slots = 4 KB of static device memory, held
-//     by every GPU that loads the library until the process exits.
+//   - The scratch is 5 KB of static device memory (1024 32-bit partial slots and one scale
+//     record), held by every GPU that loads the library until the process exits.
 //   - A call needs one slot per CTA of the amax pass; on GPUs with up to 256 SMs every shape
 //     fits.  A launch that would need more slots is rejected with NVFP4_ERR_UNSUPPORTED and a
 //     message in nvfp4_last_error(); a failed CUDA call returns NVFP4_ERR_CUDA, likewise.
 //   - All calls share the one array and it keeps the last call's contents.  Nothing in it needs
-//     to start at zero: each call's amax pass writes every slot its quantize pass reads.  Calls
+//     to start at zero: each call's amax pass writes every slot its record kernel reads, and the
+//     record kernel writes the whole record its quantize pass reads.  Calls
 //     whose kernels overlap on the GPU (different streams without ordering, several host
 //     threads) race on the array and give wrong results; order them on one stream.
 //   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
@@ -31,15 +32,16 @@ namespace {
 
 constexpr int kNoAllocPartials = 1024;
 static_assert(kNoAllocPartials >= kMaxPartials, "scratch must hold a full amax pass");
+static_assert(kNoAllocPartials * sizeof(uint32_t) == kRecordOffset, "partials, then the record");
 
-static __device__ __align__(256) uint32_t g_noalloc_partials[kNoAllocPartials];
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kTensorScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-uint32_t *g_scratch_ptr[kMaxDevices] = {nullptr};
+uint8_t *g_scratch_ptr[kMaxDevices] = {nullptr};
 
 // Device address of the scratch array on the current device (looked up once per device).
-cudaError_t scratch_for_current_device(uint32_t **out) {
+cudaError_t scratch_for_current_device(uint8_t **out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -47,9 +49,9 @@ cudaError_t scratch_for_current_device(uint32_t **out) {
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
     if (!g_scratch_ptr[dev]) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = static_cast<uint32_t *>(p);
+        g_scratch_ptr[dev] = static_cast<uint8_t *>(p);
     }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
@@ -74,6 +76,7 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, in
     const int64_t orows = dir == NVFP4_ROWWISE ? M : K, ocols = dir == NVFP4_ROWWISE ? K : M;
     if (out->rows != orows || out->cols != ocols) return NVFP4_ERR_INVALID_ARG;
     if (!aligned16(x_bf16) || (ld & 7) || (K & 7)) return NVFP4_ERR_UNSUPPORTED;
+    if ((uint64_t)(M + 128) * (uint64_t)(K + 128) >= (1ull << 35)) return NVFP4_ERR_UNSUPPORTED;   // 32-bit unit indexing
     if (dir == NVFP4_ROWWISE && (K & 15)) return NVFP4_ERR_UNSUPPORTED;
     if (!aligned16(out->codes)) return NVFP4_ERR_UNSUPPORTED;
     int dev = 0, major = 0, minor = 0;
@@ -92,7 +95,7 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, in
         record_error(msg);
         return NVFP4_ERR_UNSUPPORTED;
     }
-    uint32_t *scratch = nullptr;
+    uint8_t *scratch = nullptr;
     cudaError_t e = scratch_for_current_device(&scratch);
     if (e != cudaSuccess) {
         char msg[160];
@@ -114,13 +117,19 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, in
     j.pitch = 16 * ceil_div(ocols, 32);
     j.sf = out->sf;
     j.sf_layout = out->sf_layout;
-    j.g_out = out->g;
-    j.amax_in = nullptr;
-    j.partial = scratch;
+    j.partial = reinterpret_cast<uint32_t *>(scratch);
+    j.rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
+    RecJobs rj{};
+    rj.njobs = 1;
+    rj.npartial = npartial;
+    rj.job[0].partial = j.partial;
+    rj.job[0].amax_in = nullptr;
+    rj.job[0].rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
+    rj.job[0].g_out[0] = out->g;
+    rj.job[0].g_out[1] = nullptr;
     e = launch_amax(jobs, dev_status, nullptr, s);
-    if (e == cudaSuccess)
-        e = dir == NVFP4_ROWWISE ? launch_quantize_rows(jobs, dev_status, s)
-                                 : launch_quantize_cols(j, jobs.npartial, dev_status, s);
+    if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+    if (e == cudaSuccess) e = dir == NVFP4_ROWWISE ? launch_quantize_rows(jobs, s) : launch_quantize_cols(j, s);
     if (e != cudaSuccess) {
         char msg[160];
         std::snprintf(msg, sizeof(msg), "nvfp4_quantize_noalloc: %s", cudaGetErrorString(e));

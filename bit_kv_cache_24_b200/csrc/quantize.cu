@@ -1,16 +1,32 @@
-// quantize.cu -- BF16 -> NVFP4 quantizer kernels (HBM-bound): per-tensor amax, row-wise
-// quantization (16-blocks along the contiguous dim) and column-wise quantization (16-blocks
-// along the token dim, i.e. the row-wise quantization of the transpose).
+// quantize.cu -- BF16 -> NVFP4 quantizer kernels (HBM-bound): per-tensor amax, the per-tensor
+// scale record, row-wise quantization (16-blocks along the contiguous dim) and column-wise
+// quantization (16-blocks along the token dim, i.e. the row-wise quantization of the transpose).
 //
 // Method: LongLive-2.0 quantizes activations and weights to NVFP4 for its W4A4 linear layers
 // and its NVFP4 training GEMMs (abstract, fugumt.com mirror); the numeric steps are those of
 // the published NVFP4 format (see include/nvfp4.h).
 //
-// Design (B200): 16-byte coalesced loads, one warp covers 256 contiguous elements of a row
-// (8 per lane, a 16-block per lane pair, block max by one shuffle), packed 4-byte code stores
-// (a warp writes 128 contiguous bytes).  The amax pass writes one partial maximum per CTA
-// (BF16 magnitude bits, so the reduction is an integer max and deterministic); every CTA of the
-// quantize pass reduces the partials itself, so no atomics, memsets or grid barriers are needed.
+// Design (B200).  One quantization is three launches chained with programmatic dependent launch
+// (each kernel waits for its predecessor before touching global memory, so the next kernel's
+// launch and prologue overlap the previous one's tail):
+//   1. amax pass: 32-byte loads, 128 bytes in flight per thread; one partial maximum per CTA as
+//      BF16 magnitude bits (an integer max: deterministic, no atomics, no memset).
+//   2. scale record (one CTA per tensor): reduces the partials and writes g, den = 6g, RN(1/den)
+//      and the table r_tab[sf] = 1/(e4m3(sf) * g) of the 128 possible scale bytes.  Doing this
+//      once instead of in every CTA of the quantize pass took ~3 us and ~17% of the
+//      instructions off a 4680 x 3072 quantization.
+//   3. quantize pass: the quantizers are issue-bound (~100 instructions per 16-block before this
+//      design), so the block step is written for instruction count: a paired BF16 abs-max tree,
+//      the scale quotient b/den by one correction step on b * RN(1/den) (exact, see
+//      block_scale), 1/d from the record's table, paired FP32 multiplies and the hardware E2M1
+//      conversion.
+// Row-wise, a thread owns four consecutive 16-blocks of one row (four 32-byte loads), stores
+// its 32 code bytes as two 16-byte stores and its four scales as one 32-bit word (adjacent in
+// the tensor-core layout).  Measured alternatives that were slower on 4680 x 3072 .. 37440 x
+// 3072: a persistent kernel with a per-thread cp.async ring, a warp-specialized kernel fed by
+// bulk (TMA) copies (16 consumer warps per SM are too few to hide the block step's dependent
+// chains), one 16-block per thread, 128-thread CTAs, and a single cooperative launch with a
+// grid-wide amax.
 #include "common.cuh"
 #include "launch.h"
 
@@ -20,8 +36,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kAmaxUnroll = 8;     // 16-byte loads in flight per lane in the amax pass
-constexpr int kRowGroup = 4;       // 256-element segments a warp quantizes per iteration
+constexpr int kAmaxBytes = 128;    // bytes in flight per thread in the amax pass
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
     uint4 v;
@@ -30,76 +45,146 @@ __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
     return v;
 }
 
+// 16 or 32 bytes (8 or 16 BF16) of one row.
+template <int kWords>
+struct Unit {
+    uint32_t w[kWords];
+};
+
+template <int kWords>
+__device__ __forceinline__ Unit<kWords> ldg_unit(const uint16_t *p) {
+    Unit<kWords> u;
+    if constexpr (kWords == 8) {
+        asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(u.w[0]), "=r"(u.w[1]), "=r"(u.w[2]), "=r"(u.w[3]),
+                       "=r"(u.w[4]), "=r"(u.w[5]), "=r"(u.w[6]), "=r"(u.w[7]) : "l"(p));
+    } else {
+        const uint4 v = ldg_nc_v4(p);
+        u.w[0] = v.x; u.w[1] = v.y; u.w[2] = v.z; u.w[3] = v.w;
+    }
+    return u;
+}
+
+__device__ __forceinline__ void stg_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ uint32_t warp_max(uint32_t v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
     return v;
 }
 
-// Block-wide reduction of the amax partials of one job; returns BF16 magnitude bits, or
-// 0xFFFFFFFF when the input held inf/NaN.  Called by all threads.
-__device__ uint32_t reduce_partials(const uint32_t *partial, int n, uint32_t *smem_slot) {
-    if (threadIdx.x < 32) {
-        uint32_t m = 0;
-        for (int i = threadIdx.x; i < n; i += 32) m = max(m, partial[i]);
-        m = warp_max(m);
-        if (threadIdx.x == 0) *smem_slot = m;
+// Block-wide max of n <= kMaxPartials partials (BF16 magnitude bits).  Called by all kThreads
+// threads; red: kWarps words of shared memory.
+__device__ uint32_t reduce_partials(const uint32_t *partial, int n, uint32_t *red) {
+    constexpr int kPer = kMaxPartials / kThreads;
+    uint32_t m = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int k = threadIdx.x + i * kThreads;
+        m = max(m, k < n ? partial[k] : 0u);
     }
+    m = warp_max(m);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
-    uint32_t m = *smem_slot;
-    return m >= 0x7F80u ? 0xFFFFFFFFu : m;
+    m = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) m = max(m, red[w]);
+    return m;
+}
+static_assert(kMaxPartials % kThreads == 0, "partials split evenly over the threads");
+
+// The per-tensor scale record in shared memory, loaded by every quantize CTA.
+struct SmemRecord {
+    float r_tab[128];
+    float den, inv_den;
+    uint32_t ok;
+};
+
+// Copy the record to shared memory (after griddep_wait); a barrier must follow.
+__device__ __forceinline__ void load_record(const ScaleRecord *rec, SmemRecord &s) {
+    if (threadIdx.x < 128) s.r_tab[threadIdx.x] = rec->r_tab[threadIdx.x];
+    if (threadIdx.x == 128) {
+        s.den = rec->den;
+        s.inv_den = rec->inv_den;
+        s.ok = rec->ok;
+    }
 }
 
-// amax of one job -> g (and the non-finite check).  Returns false (after reporting) on inf/NaN.
-__device__ bool job_scale(const RowJob &j, int npartial, int32_t *status, uint32_t *smem_slot,
-                          float &g, float &den) {
-    float amax;
-    if (j.amax_in) {
-        amax = *j.amax_in;
-        if (!isfinite(amax)) {
-            if (threadIdx.x == 0) set_status(status, NVFP4_ERR_NONFINITE);
-            return false;
-        }
+// ---- the 16-block step --------------------------------------------------------------------------
+//
+// sf = e4m3(RN(b / den)).  The quotient comes from q0 = RN(b * y), y = RN(1/den), corrected once:
+// q = RN(q0 + RN(b - q0 * den) * y) with both steps fused multiply-adds.  This is the last step of
+// Markstein's division and returns RN(b/den) exactly as long as the residual b - q0*den does not
+// underflow; b >= 2^-100 and den >= 2^-125 (where y is stored nonzero) keep it normal, and every
+// other case takes the IEEE division.  (An exhaustive host-side check over all positive finite
+// BF16 b and ~800 den values, quotients up to 448, found no difference.)  r = 1/d comes from the
+// record's table; d == 0 gives r == 0, meaning every code of the block is +0.
+__device__ __forceinline__ BlockScale block_scale(float b, const SmemRecord &rec) {
+    BlockScale s;
+    float q;
+    if (b >= 0x1p-100f && rec.inv_den != 0.0f) {
+        const float q0 = __fmul_rn(b, rec.inv_den);
+        q = __fmaf_rn(__fmaf_rn(-q0, rec.den, b), rec.inv_den, q0);
     } else {
-        uint32_t bits = reduce_partials(j.partial, npartial, smem_slot);
-        if (bits == 0xFFFFFFFFu) {
-            if (threadIdx.x == 0) set_status(status, NVFP4_ERR_NONFINITE);
-            return false;
-        }
-        amax = __uint_as_float(bits << 16);
+        q = __fdiv_rn(b, rec.den);
     }
-    g = global_scale(amax);
-    den = __fmul_rn(g, kE2M1Max);
-    return true;
+    s.sf = (b == 0.0f) ? 0u : e4m3(q);
+    s.r = rec.r_tab[s.sf];
+    s.r_inf = isinf(s.r);
+    return s;
+}
+
+__device__ __forceinline__ void quantize16(const uint32_t w[8], const SmemRecord &rec,
+                                           uint32_t &c0, uint32_t &c1, uint32_t &sf) {
+    const uint32_t bm = absmax_bits16(w);
+    const BlockScale s = block_scale(__uint_as_float(bm << 16), rec);
+    sf = s.sf;
+    c0 = c1 = 0;
+    if (s.r != 0.0f) {
+        c0 = encode8(w, s);
+        c1 = encode8(w + 4, s);
+    }
 }
 
 // ---------------------------------------------------------------------------------------------
 // Pass 1: per-CTA partial max of |x| as BF16 magnitude bits (inf/NaN compare above 0x7F80).
+// A unit index maps to (row, unit in row) by one 32-bit division unless the rows are contiguous.
+template <int kWords>
 __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const __grid_constant__ RowJobs jobs) {
+    griddep_wait();
+    griddep_launch_dependents();
     const RowJob &j = jobs.job[blockIdx.y];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t cpr = j.cols >> 3;                      // 8-element chunks per row
+    constexpr int kElems = 2 * kWords;
+    constexpr int kUnroll = kAmaxBytes / (4 * kWords);
+    const uint32_t upr = (uint32_t)(j.cols / kElems);    // units per row (cols % kElems == 0)
+    const uint32_t total = (uint32_t)j.rows * upr;         // < 2^31 (checked by the host)
+    const bool flat = j.ld == j.cols;
+    const uint32_t stride = gridDim.x * kThreads;
     uint32_t m = 0;
-    for (int64_t row = (int64_t)blockIdx.x * kWarps + warp; row < j.rows; row += (int64_t)gridDim.x * kWarps) {
-        const uint16_t *xr = j.x + row * j.ld;
-        int64_t c = lane;
-        for (; c + 32 * (kAmaxUnroll - 1) < cpr; c += 32 * kAmaxUnroll) {   // kAmaxUnroll loads in flight
-            uint4 v[kAmaxUnroll];
+    for (uint32_t u0 = blockIdx.x * kThreads + threadIdx.x; u0 < total; u0 += stride * kUnroll) {
+        Unit<kWords> v[kUnroll];
 #pragma unroll
-            for (int u = 0; u < kAmaxUnroll; ++u) v[u] = ldg_nc_v4(xr + 8 * (c + 32 * u));
+        for (int k = 0; k < kUnroll; ++k) {
+            const uint32_t u = u0 + (uint32_t)k * stride;
+            if (u < total) {
+                const uint32_t row = flat ? 0u : u / upr;
+                const int64_t off = flat ? (int64_t)u * kElems : (int64_t)row * j.ld + (int64_t)(u - row * upr) * kElems;
+                v[k] = ldg_unit<kWords>(j.x + off);
+            } else {
 #pragma unroll
-            for (int u = 0; u < kAmaxUnroll; ++u) {
-                const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-                m = max(m, absmax_bits8(w));
+                for (int i = 0; i < kWords; ++i) v[k].w[i] = 0;
             }
         }
-        for (; c < cpr; c += 32) {
-            uint4 v = ldg_nc_v4(xr + 8 * c);
-            uint32_t w[4] = {v.x, v.y, v.z, v.w};
-            m = max(m, absmax_bits8(w));
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+#pragma unroll
+            for (int i = 0; i < kWords; i += 4) m = max(m, absmax_bits8(v[k].w + i));
         }
     }
     __shared__ uint32_t red[kWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     m = warp_max(m);
     if (lane == 0) red[warp] = m;
     __syncthreads();
@@ -110,12 +195,14 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const __grid_con
     }
 }
 
-// Final step of nvfp4_amax: partials -> amax float (one CTA).
-__global__ void amax_finish_kernel(const uint32_t *partial, int n, float *amax_out, int32_t *status) {
-    __shared__ uint32_t slot;
-    uint32_t bits = reduce_partials(partial, n, &slot);
+// nvfp4_amax's final step: partials -> amax float (one CTA).
+__global__ void __launch_bounds__(kThreads) amax_finish_kernel(const uint32_t *partial, int n, float *amax_out, int32_t *status) {
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ uint32_t red[kWarps];
+    const uint32_t bits = reduce_partials(partial, n, red);
     if (threadIdx.x == 0) {
-        if (bits == 0xFFFFFFFFu) {
+        if (bits >= 0x7F80u) {
             set_status(status, NVFP4_ERR_NONFINITE);
             *amax_out = __uint_as_float(0x7FC00000u);
         } else {
@@ -124,134 +211,174 @@ __global__ void amax_finish_kernel(const uint32_t *partial, int n, float *amax_o
     }
 }
 
-// ---------------------------------------------------------------------------------------------
-// Pass 2, row-wise.  Work item = (row, 256-element segment); rows are extended to a multiple of
-// 128 for the tensor-core scale layout so that its padding rows get zero scales.  Loads outside
-// the matrix read as zero, which quantizes to zero codes and zero scales: that writes every
-// padding byte of codes (to a multiple of 32 elements) and scales (to a multiple of 64).
-__global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_constant__ RowJobs jobs, int32_t *status) {
-    const RowJob j = jobs.job[blockIdx.y];
-    __shared__ uint32_t slot;
-    float g, den;
-    if (!job_scale(j, jobs.npartial, status, &slot, g, den)) return;
-    if (blockIdx.x == 0 && threadIdx.x == 0) *j.g_out = g;
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const bool mma = j.sf_layout != 0;
-    const int64_t nb = ceil_div(j.cols, 16);
-    const int64_t nb_pad = mma ? 4 * ceil_div(nb, 4) : nb;
-    const int64_t atoms = ceil_div(nb, 4);
-    const int64_t code_cols = 32 * ceil_div(j.cols, 32);
-    const int64_t rows_total = mma ? 128 * ceil_div(j.rows, 128) : j.rows;
-    const int64_t nseg = ceil_div(mma ? 16 * nb_pad : code_cols, 256);
-    const int64_t ngrp = ceil_div(nseg, kRowGroup);
-    const int64_t items = rows_total * ngrp;
-
-    for (int64_t it = (int64_t)blockIdx.x * kWarps + warp; it < items; it += (int64_t)gridDim.x * kWarps) {
-        const int64_t row = it / ngrp;
-        const int64_t e0 = (it - row * ngrp) * (256 * kRowGroup) + lane * 8;
-        uint4 v[kRowGroup];
-#pragma unroll
-        for (int u = 0; u < kRowGroup; ++u) {           // all loads of the group first
-            const int64_t e = e0 + 256 * u;
-            v[u] = make_uint4(0, 0, 0, 0);
-            if (row < j.rows && e < j.cols) v[u] = ldg_nc_v4(j.x + row * j.ld + e);
+// Pass 2: the scale record of each tensor (one CTA per job) from its partials or its amax_in.
+__global__ void __launch_bounds__(kThreads) scale_record_kernel(const __grid_constant__ RecJobs jobs, int32_t *status) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const RecJob &j = jobs.job[blockIdx.x];
+    __shared__ uint32_t red[kWarps];
+    float amax;
+    bool finite;
+    if (j.amax_in) {
+        amax = *j.amax_in;
+        finite = isfinite(amax);
+    } else {
+        const uint32_t bits = reduce_partials(j.partial, jobs.npartial, red);
+        finite = bits < 0x7F80u;
+        amax = __uint_as_float(bits << 16);
+    }
+    ScaleRecord *rec = j.rec;
+    if (!finite) {
+        if (threadIdx.x == 0) {
+            rec->ok = 0;
+            set_status(status, NVFP4_ERR_NONFINITE);
         }
+        return;
+    }
+    const float g = global_scale(amax);
+    const float den = __fmul_rn(g, kE2M1Max);
+    if (threadIdx.x < 128) {
+        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
+        rec->r_tab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+    }
+    if (threadIdx.x == 128) {
+        rec->g = g;
+        rec->den = den;
+        rec->inv_den = den >= 0x1p-125f ? __frcp_rn(den) : 0.0f;
+        rec->ok = 1;
+        if (j.g_out[0]) *j.g_out[0] = g;
+        if (j.g_out[1]) *j.g_out[1] = g;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Pass 3, row-wise (cols % 16 == 0).  A thread owns quad (row, q): 16-blocks 4q..4q+3 of a row,
+// 64 elements.  Rows run to a multiple of 128 in the tensor-core scale layout, whose padding rows
+// get zero scales (no loads, no codes); blocks past the row's end quantize to zero codes and
+// scales, which writes the code padding (to a multiple of 32 elements) and the scale padding
+// (to a multiple of 64) of the tensor-core layout.
+template <bool kV8, bool kMma>
+__global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_constant__ RowJobs jobs) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const RowJob &j = jobs.job[blockIdx.y];
+    __shared__ SmemRecord rec;
+    const uint32_t rows = (uint32_t)j.rows;
+    const uint32_t nb = (uint32_t)(j.cols >> 4);            // 16-blocks per row
+    const uint32_t nq = (nb + 3) >> 2;                      // quads per row
+    const uint32_t rows_total = kMma ? 128u * ((rows + 127u) >> 7) : rows;
+    const uint32_t idx = blockIdx.x * kThreads + threadIdx.x;
+    const bool active = idx < rows_total * nq;              // < 2^31 (checked by the host)
+    const uint32_t row = active ? idx / nq : 0u;
+    const uint32_t q = idx - row * nq;
+    const bool live = active && row < rows;                 // a row of x (not scale padding)
+
+    uint32_t w[4][8];
+    const uint16_t *xr = j.x + (int64_t)row * j.ld + 64 * q;
 #pragma unroll
-        for (int u = 0; u < kRowGroup; ++u) {
-            const int64_t e = e0 + 256 * u;
-            if (e >= nseg * 256) break;                 // past the last segment (warp-uniform)
-            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-            uint32_t bm = absmax_bits8(w);
-            bm = max(bm, __shfl_xor_sync(0xFFFFFFFFu, bm, 1));
-            const BlockScale sc = block_scale(__uint_as_float(bm << 16), g, den);
-            const uint32_t codes = (sc.r == 0.0f) ? 0u : encode8(w, sc);
-            if (row < j.rows && e < code_cols)
-                *reinterpret_cast<uint32_t *>(j.codes + row * j.pitch + (e >> 1)) = codes;
-            if ((lane & 1) == 0) {
-                const int64_t blk = e >> 4;
-                if (!mma) {
-                    if (row < j.rows && blk < nb) j.sf[row * nb + blk] = (uint8_t)sc.sf;
-                } else if (blk < nb_pad) {
-                    j.sf[sf_mma_offset(row, blk, atoms)] = (uint8_t)sc.sf;
-                }
+    for (int b = 0; b < 4; ++b) {
+        if (live && 4 * q + b < nb) {
+            if constexpr (kV8) {
+                const Unit<8> u = ldg_unit<8>(xr + 16 * b);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) w[b][i] = u.w[i];
+            } else {
+                const uint4 u0 = ldg_nc_v4(xr + 16 * b), u1 = ldg_nc_v4(xr + 16 * b + 8);
+                w[b][0] = u0.x; w[b][1] = u0.y; w[b][2] = u0.z; w[b][3] = u0.w;
+                w[b][4] = u1.x; w[b][5] = u1.y; w[b][6] = u1.z; w[b][7] = u1.w;
             }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[b][i] = 0;
+        }
+    }
+    load_record(j.rec, rec);
+    __syncthreads();
+    if (!active || !rec.ok) return;
+
+    uint32_t c[8], sfw = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        uint32_t sf;
+        quantize16(w[b], rec, c[2 * b], c[2 * b + 1], sf);
+        sfw |= sf << (8 * b);
+    }
+    if (live) {
+        uint8_t *cr = j.codes + (int64_t)row * j.pitch + 32 * q;
+        if (32 * q < j.pitch) stg_v4(cr, c[0], c[1], c[2], c[3]);
+        if (32 * q + 16 < j.pitch) stg_v4(cr + 16, c[4], c[5], c[6], c[7]);
+    }
+    if constexpr (kMma) {
+        *reinterpret_cast<uint32_t *>(j.sf + sf_mma_offset(row, 4 * q, nq)) = sfw;
+    } else if (live) {
+        uint8_t *sr = j.sf + (int64_t)row * nb + 4 * q;
+        if (4 * q + 3 < nb && ((reinterpret_cast<uintptr_t>(sr) & 3) == 0)) {
+            *reinterpret_cast<uint32_t *>(sr) = sfw;
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                if (4 * q + b < nb) sr[b] = (uint8_t)(sfw >> (8 * b));
         }
     }
 }
 
 // ---------------------------------------------------------------------------------------------
-// Pass 2, column-wise: 16-blocks along the rows (m) of x [M][K]; output row k holds x[:, k].
-// A CTA stages a 256 (m) x 32 (k) BF16 tile in shared memory (16 KB), words XOR-swizzled by the
-// 16-row group so that the 16 threads reading one k down 16 different m-blocks hit 16 banks.
-// Thread (k, m-block) then quantizes 16 values; lanes 0-15 of a warp share k, so a warp writes
-// 128 contiguous code bytes per output row.
-constexpr int kColTileM = 256, kColTileK = 32;
-
-__global__ void __launch_bounds__(kThreads) quantize_cols_kernel(RowJob j, int32_t npartial, int32_t *status) {
-    __shared__ uint32_t tile[kColTileM * (kColTileK / 2)];
-    __shared__ uint32_t slot;
-    float g, den;
-    if (!job_scale(j, npartial, status, &slot, g, den)) return;
-    if (blockIdx.x == 0 && threadIdx.x == 0) *j.g_out = g;
-
+// Pass 3, column-wise: 16-blocks along the rows (m) of x [M][K]; output row k holds x[:, k].
+// Transpose in registers: a thread loads a 16 (m) x 8 (k) patch (sixteen 16-byte row pieces, all
+// in flight at once) and emits the eight 16-blocks of its eight columns.  Lanes 0-7 of a warp
+// take adjacent 8-column chunks (a full 128-byte line of each row) and lane groups 0-3 adjacent
+// 16-row blocks, so a warp covers 64 x 64 and each 8-byte code store instruction writes eight
+// output rows x 32 contiguous bytes.  Output rows run to a multiple of 128 and scale columns to
+// a multiple of 4 in the tensor-core layout (zero scales); code columns run to a multiple of 32.
+__global__ void __launch_bounds__(kThreads) quantize_cols_kernel(const __grid_constant__ RowJob j) {
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ SmemRecord rec;
     const bool mma = j.sf_layout != 0;
-    const int64_t M = j.rows, K = j.cols;                 // x is [M][K]; output is [K][M]
-    const int64_t nb = ceil_div(M, 16);                   // scale columns of the output
-    const int64_t nb_pad = mma ? 4 * ceil_div(nb, 4) : nb;
-    const int64_t atoms = ceil_div(nb, 4);
-    const int64_t code_cols = 32 * ceil_div(M, 32);
-    const int64_t m_extent = mma ? 16 * nb_pad : code_cols;
-    const int64_t k_extent = mma ? 128 * ceil_div(K, 128) : K;
-    const int64_t tiles_m = ceil_div(m_extent, kColTileM), tiles_k = ceil_div(k_extent, kColTileK);
-    const int t = threadIdx.x;
+    const uint32_t M = (uint32_t)j.rows, K = (uint32_t)j.cols;   // x is [M][K]; output is [K][M]
+    const uint32_t nb = (M + 15) >> 4;                      // scale columns of the output
+    const uint32_t nb_pad = mma ? 4 * ((nb + 3) >> 2) : nb;
+    const uint32_t atoms = (nb + 3) >> 2;
+    const uint32_t code_cols = 32 * ((M + 31) >> 5);
+    const uint32_t mb_total = (mma ? 16 * nb_pad : code_cols) >> 4;   // 16-row blocks to cover
+    const uint32_t k_extent = mma ? 128 * ((K + 127) >> 7) : K;
+    const uint32_t kc_total = k_extent >> 3;                // 8-column chunks (K % 8 == 0)
+    const uint32_t tiles_k = (kc_total + 7) >> 3, tiles_m = (mb_total + 3) >> 2;
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t wt = blockIdx.x * kWarps + (threadIdx.x >> 5);      // warp tile, k fastest
+    const bool active = wt < tiles_k * tiles_m;
+    const uint32_t tk = active ? wt % tiles_k : 0u, tm = active ? wt / tiles_k : 0u;
+    const uint32_t kc = 8 * tk + (lane & 7), mb = 4 * tm + (lane >> 3);
+    const uint32_t k0 = 8 * kc, m0 = 16 * mb;
 
-    for (int64_t tile_id = blockIdx.x; tile_id < tiles_m * tiles_k; tile_id += gridDim.x) {
-        const int64_t m0 = (tile_id % tiles_m) * kColTileM, k0 = (tile_id / tiles_m) * kColTileK;
-        __syncthreads();                                  // previous tile fully consumed
-        // load: thread t covers rows t/4 + 64*i, 8-element chunk t%4 of the 32 k
+    uint32_t w[16][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = (t >> 2) + 64 * i, c = t & 3;
-            const int64_t m = m0 + r, k = k0 + 8 * c;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (m < M && k < K) v = ldg_nc_v4(j.x + m * j.ld + k);
-            const int swz = (r >> 4) & 15;
-            uint32_t *row = tile + r * (kColTileK / 2);
-            row[(4 * c + 0) ^ swz] = v.x;
-            row[(4 * c + 1) ^ swz] = v.y;
-            row[(4 * c + 2) ^ swz] = v.z;
-            row[(4 * c + 3) ^ swz] = v.w;
-        }
-        __syncthreads();
+    for (int r = 0; r < 16; ++r) {
+        const uint32_t m = m0 + r;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (active && m < M && k0 < K) v = ldg_nc_v4(j.x + (int64_t)m * j.ld + k0);
+        w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
+    }
+    load_record(j.rec, rec);
+    __syncthreads();
+    if (!active || !rec.ok || kc >= kc_total || mb >= mb_total) return;
+
 #pragma unroll
-        for (int p2 = 0; p2 < 2; ++p2) {
-            const int p = t + kThreads * p2;
-            const int kl = p >> 4, mb = p & 15;           // local k row, local 16-block
-            const int shift = (kl & 1) * 16;
-            uint32_t w[8];
+    for (int c = 0; c < 4; ++c) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int r0 = mb * 16 + 2 * i, r1 = r0 + 1;
-                const uint32_t a = tile[r0 * (kColTileK / 2) + ((kl >> 1) ^ mb)] >> shift;
-                const uint32_t b = tile[r1 * (kColTileK / 2) + ((kl >> 1) ^ mb)] >> shift;
-                w[i] = (a & 0xFFFFu) | (b << 16);
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t k = k0 + 2 * c + h;
+            uint32_t b[8];                                   // column k, rows m0..m0+15 as BF16 pairs
+#pragma unroll
+            for (int i = 0; i < 8; ++i) b[i] = __byte_perm(w[2 * i][c], w[2 * i + 1][c], h ? 0x7632 : 0x5410);
+            uint32_t c0, c1, sf;
+            quantize16(b, rec, c0, c1, sf);
+            if (k < K) {
+                if (m0 < code_cols)
+                    *reinterpret_cast<uint2 *>(j.codes + (int64_t)k * j.pitch + (m0 >> 1)) = make_uint2(c0, c1);
+                if (!mma && mb < nb) j.sf[(int64_t)k * nb + mb] = (uint8_t)sf;
             }
-            const uint32_t bm = max(absmax_bits8(w), absmax_bits8(w + 4));
-            const BlockScale s = block_scale(__uint_as_float(bm << 16), g, den);
-            uint2 codes = make_uint2(0, 0);
-            if (s.r != 0.0f) {
-                codes.x = encode8(w, s);
-                codes.y = encode8(w + 4, s);
-            }
-            const int64_t k = k0 + kl, m = m0 + 16 * mb, blk = m >> 4;
-            if (k < K && m < code_cols)
-                *reinterpret_cast<uint2 *>(j.codes + k * j.pitch + (m >> 1)) = codes;
-            if (!mma) {
-                if (k < K && blk < nb) j.sf[k * nb + blk] = (uint8_t)s.sf;
-            } else if (k < k_extent && blk < nb_pad) {
-                j.sf[sf_mma_offset(k, blk, atoms)] = (uint8_t)s.sf;
-            }
+            if (mma) j.sf[sf_mma_offset(k, mb, atoms)] = (uint8_t)sf;
         }
     }
 }
@@ -283,48 +410,57 @@ __global__ void wait_timeout_kernel(int32_t *status, int64_t limit_ns) {
     }
 }
 
+bool all_v8(const RowJobs &jobs) {
+    for (int i = 0; i < jobs.njobs; ++i) {
+        const RowJob &j = jobs.job[i];
+        if ((reinterpret_cast<uintptr_t>(j.x) & 31) || (j.ld & 15) || (j.cols & 15)) return false;
+    }
+    return true;
+}
+
 }  // namespace
 
 int amax_blocks(int64_t rows) {
-    int64_t b = ceil_div(rows, kWarps);
-    const int64_t cap = 6 * (int64_t)num_sms();          // 6 x 256 threads per SM
-    if (b > cap) b = cap;
-    if (b > kMaxPartials) b = kMaxPartials;
-    return (int)(b < 1 ? 1 : b);
+    (void)rows;
+    return 4 * num_sms() < kMaxPartials ? 4 * num_sms() : kMaxPartials;   // 4 x 256 threads per SM
 }
 
 cudaError_t launch_amax(const RowJobs &jobs, int32_t *status, float *amax_out, cudaStream_t s) {
-    dim3 grid(jobs.npartial, jobs.njobs);
-    amax_partial_kernel<<<grid, kThreads, 0, s>>>(jobs);
-    if (amax_out) amax_finish_kernel<<<1, 32, 0, s>>>(jobs.job[0].partial, jobs.npartial, amax_out, status);
-    return cudaGetLastError();
+    const dim3 grid(jobs.npartial, jobs.njobs);
+    cudaError_t e = all_v8(jobs) ? launch_pdl(amax_partial_kernel<8>, grid, dim3(kThreads), 0, s, jobs)
+                                 : launch_pdl(amax_partial_kernel<4>, grid, dim3(kThreads), 0, s, jobs);
+    if (e == cudaSuccess && amax_out)
+        e = launch_pdl(amax_finish_kernel, dim3(1), dim3(kThreads), 0, s,
+                       (const uint32_t *)jobs.job[0].partial, (int)jobs.npartial, amax_out, status);
+    return e;
 }
 
-cudaError_t launch_quantize_rows(const RowJobs &jobs, int32_t *status, cudaStream_t s) {
-    int64_t items = 0;
+cudaError_t launch_scale_record(const RecJobs &jobs, int32_t *status, cudaStream_t s) {
+    return launch_pdl(scale_record_kernel, dim3(jobs.njobs), dim3(kThreads), 0, s, jobs, status);
+}
+
+cudaError_t launch_quantize_rows(const RowJobs &jobs, cudaStream_t s) {
+    int64_t quads = 0;
     for (int i = 0; i < jobs.njobs; ++i) {
         const RowJob &j = jobs.job[i];
         const int64_t rows = j.sf_layout ? 128 * ceil_div(j.rows, 128) : j.rows;
-        const int64_t it = rows * ceil_div(ceil_div(64 * ceil_div(j.cols, 64), 256), kRowGroup);
-        if (it > items) items = it;
+        const int64_t n = rows * ceil_div(j.cols / 16, 4);
+        if (n > quads) quads = n;
     }
-    int64_t blocks = ceil_div(items, kWarps);
-    const int64_t cap = 8 * (int64_t)num_sms();            // 8 x 256 threads fill an SM
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
-    quantize_rows_kernel<<<dim3((unsigned)blocks, jobs.njobs), kThreads, 0, s>>>(jobs, status);
-    return cudaGetLastError();
+    const dim3 grid((unsigned)ceil_div(quads, kThreads), jobs.njobs), block(kThreads);
+    const bool v8 = all_v8(jobs), mma = jobs.job[0].sf_layout != 0;   // jobs of one launch share the layout
+    if (v8 && mma) return launch_pdl(quantize_rows_kernel<true, true>, grid, block, 0, s, jobs);
+    if (v8) return launch_pdl(quantize_rows_kernel<true, false>, grid, block, 0, s, jobs);
+    if (mma) return launch_pdl(quantize_rows_kernel<false, true>, grid, block, 0, s, jobs);
+    return launch_pdl(quantize_rows_kernel<false, false>, grid, block, 0, s, jobs);
 }
 
-cudaError_t launch_quantize_cols(const RowJob &j, int32_t npartial, int32_t *status, cudaStream_t s) {
+cudaError_t launch_quantize_cols(const RowJob &j, cudaStream_t s) {
     const int64_t nb = ceil_div(j.rows, 16);
     const int64_t m_extent = j.sf_layout ? 64 * ceil_div(nb, 4) : 32 * ceil_div(j.rows, 32);
     const int64_t k_extent = j.sf_layout ? 128 * ceil_div(j.cols, 128) : j.cols;
-    int64_t tiles = ceil_div(m_extent, kColTileM) * ceil_div(k_extent, kColTileK);
-    const int64_t cap = 6 * (int64_t)num_sms();
-    if (tiles > cap) tiles = cap;
-    quantize_cols_kernel<<<(unsigned)tiles, kThreads, 0, s>>>(j, npartial, status);
-    return cudaGetLastError();
+    const int64_t warp_tiles = ceil_div(k_extent / 8, 8) * ceil_div(m_extent / 16, 4);
+    return launch_pdl(quantize_cols_kernel, dim3((unsigned)ceil_div(warp_tiles, kWarps)), dim3(kThreads), 0, s, j);
 }
 
 cudaError_t launch_encode_elements(const float *in, int64_t n, uint8_t *e2m1_out, uint8_t *e4m3_out, cudaStream_t s) {

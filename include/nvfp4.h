@@ -63,7 +63,7 @@ typedef enum {
     NVFP4_ERR_CUDA = 5          /* a CUDA runtime/driver call failed */
 } nvfp4_status;
 
-typedef enum { NVFP4_ROWWISE = 0, NVFP4_COLWISE = 1 } nvfp4_dir;
+typedef enum { NVFP4_ROWWISE = 0, NVFP4_COLWISE = 1, NVFP4_ROWCOL = 2 } nvfp4_dir;
 typedef enum { NVFP4_SF_LINEAR = 0, NVFP4_SF_MMA = 1 } nvfp4_sf_layout;
 typedef enum { NVFP4_OUT_BF16 = 0, NVFP4_OUT_F32 = 1 } nvfp4_out_dtype;
 
@@ -103,10 +103,11 @@ NVFP4_API int64_t nvfp4_codes_pitch(int64_t cols);
 /* Bytes of the scale array of a rows x cols matrix in `layout`; -1 on bad arguments. */
 NVFP4_API int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols, int32_t layout);
 
-/* Bytes of device workspace nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima). */
+/* Bytes of device workspace nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima and the
+ * per-tensor scale record; 5 KB). */
 NVFP4_API size_t nvfp4_quantize_workspace(int64_t rows, int64_t cols);
 
-/* Bytes of device workspace kv_quant_append needs (partial maxima of K and of V). */
+/* Bytes of device workspace kv_quant_append needs (the same, for K and for V). */
 NVFP4_API size_t nvfp4_kv_append_workspace(int64_t ntok, int32_t heads, int32_t head_dim);
 
 /* ---- the four calls of the path ------------------------------------------------------------- */
@@ -128,10 +129,14 @@ NVFP4_API nvfp4_status nvfp4_amax(const void *x_bf16, int64_t M, int64_t K, int6
  *   dir = NVFP4_COLWISE: 16-blocks along M (the token dim), i.e. the row-wise quantization of
  *         x^T, as needed for the wgrad/dgrad operands of NVFP4 training GEMMs; out->rows = K,
  *         out->cols = M; a trailing partial block (M % 16 != 0) is zero-padded.
- * amax_in: nullable DEVICE pointer to a precomputed amax of x (from nvfp4_amax); when NULL the
- * amax pass runs first (two launches).  out->g receives g; out->sf uses out->sf_layout.  All
- * padding bytes of codes and scales are written (zero).  ws: nvfp4_quantize_workspace(M, K)
- * bytes of device memory, only used when amax_in is NULL.
+ *   dir = NVFP4_ROWCOL: both layouts with one amax in one call: `out` points to two tensors,
+ *         out[0] row-wise ([M, K]) and out[1] column-wise ([K, M]).  Requires K % 16 == 0.
+ * amax_in: nullable DEVICE pointer to a precomputed amax of x (from nvfp4_amax); when NULL a
+ * first pass computes it.  out->g receives g; out->sf uses out->sf_layout.  All padding bytes of
+ * codes and scales are written (zero).  ws: nvfp4_quantize_workspace(M, K) bytes of device
+ * memory (16-byte aligned, no initialisation needed), required in every call: it holds the
+ * amax partials and the per-tensor scale record.  (M + 128) * (K + 128) must be below 2^35,
+ * else NVFP4_ERR_UNSUPPORTED.
  */
 NVFP4_API nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld, int32_t dir,
                             const float *amax_in, const nvfp4_tensor *out, void *ws,
@@ -161,7 +166,7 @@ NVFP4_API int64_t nvfp4_kv_cache_bytes(int32_t layers, int32_t heads, int32_t he
  * nothing else in the cache is touched and older slots are never re-quantized.  Each of K and V
  * gets its own per-tensor scale (g_k/g_v[layer*slots + slot]).  Sets cache->len[layer*slots +
  * slot] = ntok (host).  Requires ntok <= slot_tokens, head_dim % 16 == 0, ws of
- * nvfp4_kv_append_workspace bytes.
+ * nvfp4_kv_append_workspace bytes, (ntok + 128) * (heads * head_dim + 128) below 2^35.
  */
 NVFP4_API nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int32_t slot,
                              const void *k_bf16, const void *v_bf16, int64_t ntok, int64_t ld,
@@ -183,8 +188,8 @@ NVFP4_API nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, co
  * receive only their input and output buffers and have no allocator or workspace to hand over.
  * No counterpart in the paper: it is a deployment variant of the quantizer above.
  * Same arguments, layouts and results as nvfp4_quantize with amax_in = NULL, bit for bit; the
- * amax partial maxima go to a 4 KB (1024-slot) static device array held by every GPU that loads
- * the library.  Nothing is allocated.  A launch needing more than 1024 slots (only possible on
+ * amax partial maxima (1024 slots) and the scale record go to a 5 KB static device array held
+ * by every GPU that loads the library.  Nothing is allocated.  A launch needing more than 1024 slots (only possible on
  * GPUs with more than 256 SMs) returns NVFP4_ERR_UNSUPPORTED with a message in
  * nvfp4_last_error().  All calls share the array: calls whose kernels overlap on the GPU race
  * and must be ordered on one stream.  The first call on each device looks up the array's device

@@ -114,3 +114,31 @@ def test_full_size_ffn_down_activation(orc):
     gq = nv.nvfp4_quantize(A.cuda(), nv.ROWWISE)
     _, oq = orc.quantize(A)
     assert_quantized_equal(orc, gq, oq, "ffn down A")
+
+
+@pytest.mark.parametrize("rows,cols,kind", [(1, 16, "normal"), (37, 48, "outliers"), (300, 96, "wide"),
+                                            (1040, 512, "lognormal"), (4680, 3072, "lognormal"), (6000, 256, "normal")])
+@pytest.mark.parametrize("layout", [nv.SF_LINEAR, nv.SF_MMA])
+def test_rowcol_from_one_read(orc, rows, cols, kind, layout):
+    """NVFP4_ROWCOL: row-wise and column-wise outputs of one call equal the oracle's, byte for byte."""
+    x = synth.ragged(rows * 5 + cols, rows, cols, kind)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gr, gc = nv.nvfp4_quantize(x.cuda(), nv.ROWCOL, sf_layout=layout, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    _, orow = orc.quantize(x)
+    _, ocol = orc.quantize(x, colwise=True)
+    assert_quantized_equal(orc, gr, orow, f"rowcol-row {rows}x{cols}")
+    assert_quantized_equal(orc, gc, ocol, f"rowcol-col {rows}x{cols}")
+
+
+def test_repeated_calls_share_workspace(orc):
+    """Consecutive single-launch quantizations reuse one workspace: each launch's grid-wide amax
+    must ignore the previous launch's slots."""
+    L = nv.lib()
+    ws = torch.empty(L.nvfp4_quantize_workspace(4680, 3072), dtype=torch.uint8, device="cuda")
+    xs = [synth.ragged(40 + i, 4680, 3072, kind) for i, kind in enumerate(["lognormal", "wide", "normal"])]
+    outs = [nv.nvfp4_quantize(x.cuda(), nv.ROWWISE, ws=ws) for x in xs]
+    for x, g in zip(xs, outs):
+        _, o = orc.quantize(x)
+        assert_quantized_equal(orc, g, o, "shared ws")
