@@ -208,10 +208,11 @@ class QKVStep:
         # GEMM; K/V amax + record + row pass (both tensors per launch); dequant
         self.launches_per_step = 3 + 4 + 1 + 3 + 1
 
-    def step(self, i, events=None, A=None):
+    def step(self, i, events=None, A=None, Y=None):
         nv = self.nv
         s = self.sets[i % len(self.sets)]
         A = s["A"] if A is None else A
+        Y = self.Y if Y is None else Y
         ev = events
 
         def mark(j):
@@ -222,9 +223,9 @@ class QKVStep:
         mark(1)
         nv.nvfp4_quantize(A, nv.ROWCOL, out=(self.Aq, self.Acq), ws=self.ws_a, status=self.status)
         mark(2)
-        nv.nvfp4_gemm(self.Aq, self.Wq, bias=s["bias"], out=self.Y, status=self.status)
+        nv.nvfp4_gemm(self.Aq, self.Wq, bias=s["bias"], out=Y, status=self.status)
         mark(3)
-        nv.kv_quant_append(self.cache, 0, i % SLOTS, self.Y[:, HID:2 * HID], self.Y[:, 2 * HID:],
+        nv.kv_quant_append(self.cache, 0, i % SLOTS, Y[:, HID:2 * HID], Y[:, 2 * HID:],
                            status=self.status)
         mark(4)
         nv.kv_dequant(self.cache, 0, self.slots, k_out=self.Kout, v_out=self.Vout, status=self.status)
@@ -285,23 +286,56 @@ def run_ours(args, rank, local_rank, world):
     max_s = reduce_max(total_ms / 1e3, dist, dev)
     value = aggregate(GEMM_FLOP * K / 1e12, world, max_s)
 
-    # end to end through the public API: pinned host A -> device, the step, Y -> pinned host
+    # end to end through the public API: every step copies its A from pinned host memory to the
+    # device, runs the step and copies its Y back to pinned host memory.  The copies run on their
+    # own streams and overlap neighbouring steps' compute (double-buffered A and Y on the device),
+    # as a serving pipeline would; the timed region spans the first copy in to the last copy out.
     E = args.e2e_steps
     e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    A_dev = torch.empty_like(st.sets[0]["A"])
-    for i in range(3):
-        A_dev.copy_(st.A_host, non_blocking=True)
-        st.step(i, A=A_dev)
-        st.Y_host.copy_(st.Y, non_blocking=True)
+    A_dev = [torch.empty_like(st.sets[0]["A"]) for _ in range(2)]
+    Y_dev = [st.Y, torch.empty_like(st.Y)]
+    comp = torch.cuda.current_stream()
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def e2e_run(n, first=None, last=None):
+        a_free = [None, None]                             # compute done with A_dev[b]
+        y_free = [None, None]                             # copy-out done with Y_dev[b]
+        if first is not None:
+            first.record(comp)
+            h2d.wait_event(first)
+            d2h.wait_event(first)
+        for i in range(n):
+            b = i & 1
+            with torch.cuda.stream(h2d):
+                if a_free[b] is not None:
+                    h2d.wait_event(a_free[b])
+                A_dev[b].copy_(st.A_host, non_blocking=True)
+                a_in = torch.cuda.Event()
+                a_in.record(h2d)
+            comp.wait_event(a_in)
+            if y_free[b] is not None:
+                comp.wait_event(y_free[b])
+            st.step(i, A=A_dev[b], Y=Y_dev[b])
+            done = torch.cuda.Event()
+            done.record(comp)
+            a_free[b] = done
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done)
+                st.Y_host.copy_(Y_dev[b], non_blocking=True)
+                y_out = torch.cuda.Event()
+                y_out.record(d2h)
+            y_free[b] = y_out
+        for ev in y_free:
+            if ev is not None:
+                comp.wait_event(ev)
+        if last is not None:
+            last.record(comp)
+
+    e2e_run(3)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    e2e_ev[0].record()
-    for i in range(E):
-        A_dev.copy_(st.A_host, non_blocking=True)
-        st.step(i, A=A_dev)
-        st.Y_host.copy_(st.Y, non_blocking=True)
-    e2e_ev[1].record()
+    e2e_run(E, e2e_ev[0], e2e_ev[1])
     torch.cuda.synchronize()
     e2e_s = reduce_max(e2e_ev[0].elapsed_time(e2e_ev[1]) / 1e3, dist, dev)
     e2e = {"value": aggregate(GEMM_FLOP * E / 1e12, world, e2e_s), "unit": UNIT,
