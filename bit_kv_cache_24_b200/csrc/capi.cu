@@ -193,7 +193,7 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
         jc.pitch = codes_pitch(M);
         jc.sf = col_out->sf;
         jc.sf_layout = col_out->sf_layout;
-        e = launch_quantize_cols(jc, s);
+        e = launch_quantize_cols(jc, row_out != nullptr, s);
     }
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_quantize");
 }

@@ -29,7 +29,9 @@ constexpr float kGlobalDen = kE2M1Max * kE4M3Max;   // 2688: maps the tensor max
 // Every kernel of the library is launched with programmatic stream serialization (launch_pdl) and
 // calls griddep_wait() before its first global memory access: that returns once the preceding
 // kernel in the stream has completed and its writes are visible, so only the launch and the
-// prologue overlap the predecessor's tail.  griddep_launch_dependents() (after the wait) lets the
+// prologue overlap the predecessor's tail.  One exception, argued where it is made: the
+// column-wise pass of a both-layouts quantization runs concurrently with the row-wise pass and
+// waits at exit instead.  griddep_launch_dependents() (after the wait) lets the
 // next kernel be scheduled early.  Both are no-ops in a launch without the attribute.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }

@@ -59,8 +59,9 @@ struct RecJobs {
 cudaError_t launch_amax(const RowJobs &jobs, int32_t *status, float *amax_out, cudaStream_t s);
 cudaError_t launch_scale_record(const RecJobs &jobs, int32_t *status, cudaStream_t s);
 cudaError_t launch_quantize_rows(const RowJobs &jobs, cudaStream_t s);
-// Column-wise: blocks along the rows of x; output [cols][pitch(rows)].
-cudaError_t launch_quantize_cols(const RowJob &job, cudaStream_t s);
+// Column-wise: blocks along the rows of x; output [cols][pitch(rows)].  after_rows: launched
+// directly after launch_quantize_rows of the same x and record (runs concurrently with it).
+cudaError_t launch_quantize_cols(const RowJob &job, bool after_rows, cudaStream_t s);
 int amax_blocks(int64_t rows);
 
 // Launch with programmatic stream serialization (see griddep_wait in common.cuh).

@@ -129,7 +129,7 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, in
     rj.job[0].g_out[1] = nullptr;
     e = launch_amax(jobs, dev_status, nullptr, s);
     if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
-    if (e == cudaSuccess) e = dir == NVFP4_ROWWISE ? launch_quantize_rows(jobs, s) : launch_quantize_cols(j, s);
+    if (e == cudaSuccess) e = dir == NVFP4_ROWWISE ? launch_quantize_rows(jobs, s) : launch_quantize_cols(j, false, s);
     if (e != cudaSuccess) {
         char msg[160];
         std::snprintf(msg, sizeof(msg), "nvfp4_quantize_noalloc: %s", cudaGetErrorString(e));

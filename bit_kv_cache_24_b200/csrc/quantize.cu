@@ -6,9 +6,10 @@
 // and its NVFP4 training GEMMs (abstract, fugumt.com mirror); the numeric steps are those of
 // the published NVFP4 format (see include/nvfp4.h).
 //
-// Design (B200).  One quantization is three launches chained with programmatic dependent launch
-// (each kernel waits for its predecessor before touching global memory, so the next kernel's
-// launch and prologue overlap the previous one's tail):
+// Design (B200).  One quantization is three launches (four for both layouts) chained with
+// programmatic dependent launch (each kernel waits for its predecessor before touching global
+// memory, so the next kernel's launch and prologue overlap the previous one's tail; the column
+// pass after a row pass runs concurrently with it, see quantize_cols_kernel):
 //   1. amax pass: 32-byte loads, 128 bytes in flight per thread; one partial maximum per CTA as
 //      BF16 magnitude bits (an integer max: deterministic, no atomics, no memset).
 //   2. scale record (one CTA per tensor): reduces the partials and writes g, den = 6g, RN(1/den)
@@ -102,13 +103,28 @@ struct SmemRecord {
     uint32_t ok;
 };
 
-// Copy the record to shared memory (after griddep_wait); a barrier must follow.
+__device__ __forceinline__ uint32_t ldg_cg_u32(const void *p) {
+    uint32_t v;
+    asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ldg_cg_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+// Copy the record to shared memory (after griddep_wait, or through L2 with kL2 set); a barrier
+// must follow.
+template <bool kL2 = false>
 __device__ __forceinline__ void load_record(const ScaleRecord *rec, SmemRecord &s) {
-    if (threadIdx.x < 128) s.r_tab[threadIdx.x] = rec->r_tab[threadIdx.x];
+    if (threadIdx.x < 128)
+        s.r_tab[threadIdx.x] = kL2 ? __uint_as_float(ldg_cg_u32(rec->r_tab + threadIdx.x)) : rec->r_tab[threadIdx.x];
     if (threadIdx.x == 128) {
-        s.den = rec->den;
-        s.inv_den = rec->inv_den;
-        s.ok = rec->ok;
+        s.den = kL2 ? __uint_as_float(ldg_cg_u32(&rec->den)) : rec->den;
+        s.inv_den = kL2 ? __uint_as_float(ldg_cg_u32(&rec->inv_den)) : rec->inv_den;
+        s.ok = kL2 ? ldg_cg_u32(&rec->ok) : rec->ok;
     }
 }
 
@@ -330,10 +346,15 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_co
 // 16-row blocks, so a warp covers 64 x 64 and each 8-byte code store instruction writes eight
 // output rows x 32 contiguous bytes.  Output rows run to a multiple of 128 and scale columns to
 // a multiple of 4 in the tensor-core layout (zero scales); code columns run to a multiple of 32.
-__global__ void __launch_bounds__(kThreads) quantize_cols_kernel(const __grid_constant__ RowJob j) {
-    griddep_wait();
-    griddep_launch_dependents();
-    __shared__ SmemRecord rec;
+//
+// kConcurrent: launched right after the row pass of the same call (both layouts), whose inputs
+// it shares.  It then starts while the row pass runs: x and the scale record were complete
+// before the row pass could start (the row pass triggers its dependents only after its own
+// wait, which follows the record kernel), so the kernel reads them at once, through L2, and
+// waits for its predecessor only at exit -- every thread, so that this grid cannot complete
+// before the row pass and whatever waits on this grid also sees the row-wise outputs.
+template <bool kConcurrent>
+__device__ __forceinline__ void cols_body(const RowJob &j, SmemRecord &rec) {
     const bool mma = j.sf_layout != 0;
     const uint32_t M = (uint32_t)j.rows, K = (uint32_t)j.cols;   // x is [M][K]; output is [K][M]
     const uint32_t nb = (M + 15) >> 4;                      // scale columns of the output
@@ -356,10 +377,13 @@ __global__ void __launch_bounds__(kThreads) quantize_cols_kernel(const __grid_co
     for (int r = 0; r < 16; ++r) {
         const uint32_t m = m0 + r;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (active && m < M && k0 < K) v = ldg_nc_v4(j.x + (int64_t)m * j.ld + k0);
+        if (active && m < M && k0 < K) {
+            const uint16_t *p = j.x + (int64_t)m * j.ld + k0;
+            v = kConcurrent ? ldg_cg_v4(p) : ldg_nc_v4(p);
+        }
         w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
     }
-    load_record(j.rec, rec);
+    load_record<kConcurrent>(j.rec, rec);
     __syncthreads();
     if (!active || !rec.ok || kc >= kc_total || mb >= mb_total) return;
 
@@ -381,6 +405,15 @@ __global__ void __launch_bounds__(kThreads) quantize_cols_kernel(const __grid_co
             if (mma) j.sf[sf_mma_offset(k, mb, atoms)] = (uint8_t)sf;
         }
     }
+}
+
+template <bool kConcurrent>
+__global__ void __launch_bounds__(kThreads) quantize_cols_kernel(const __grid_constant__ RowJob j) {
+    __shared__ SmemRecord rec;
+    if constexpr (!kConcurrent) griddep_wait();
+    griddep_launch_dependents();
+    cols_body<kConcurrent>(j, rec);
+    if constexpr (kConcurrent) griddep_wait();
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -455,12 +488,14 @@ cudaError_t launch_quantize_rows(const RowJobs &jobs, cudaStream_t s) {
     return launch_pdl(quantize_rows_kernel<false, false>, grid, block, 0, s, jobs);
 }
 
-cudaError_t launch_quantize_cols(const RowJob &j, cudaStream_t s) {
+cudaError_t launch_quantize_cols(const RowJob &j, bool after_rows, cudaStream_t s) {
     const int64_t nb = ceil_div(j.rows, 16);
     const int64_t m_extent = j.sf_layout ? 64 * ceil_div(nb, 4) : 32 * ceil_div(j.rows, 32);
     const int64_t k_extent = j.sf_layout ? 128 * ceil_div(j.cols, 128) : j.cols;
     const int64_t warp_tiles = ceil_div(k_extent / 8, 8) * ceil_div(m_extent / 16, 4);
-    return launch_pdl(quantize_cols_kernel, dim3((unsigned)ceil_div(warp_tiles, kWarps)), dim3(kThreads), 0, s, j);
+    const dim3 grid((unsigned)ceil_div(warp_tiles, kWarps)), block(kThreads);
+    return after_rows ? launch_pdl(quantize_cols_kernel<true>, grid, block, 0, s, j)
+                      : launch_pdl(quantize_cols_kernel<false>, grid, block, 0, s, j);
 }
 
 cudaError_t launch_encode_elements(const float *in, int64_t n, uint8_t *e2m1_out, uint8_t *e4m3_out, cudaStream_t s) {
