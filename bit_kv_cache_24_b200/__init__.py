@@ -76,6 +76,8 @@ def lib():
             "nvfp4_quantize": (_I32, [_P, _I64, _I64, _I64, _I32, _P, ctypes.POINTER(_Tensor), _P, _SZ, _P, _P]),
             "nvfp4_quantize_noalloc": (_I32, [_P, _I64, _I64, _I64, _I32, ctypes.POINTER(_Tensor), _P, _P]),
             "nvfp4_gemm": (_I32, [ctypes.POINTER(_Tensor), ctypes.POINTER(_Tensor), _P, _P, _P, _I64, _I32, _P, _P]),
+            "nvfp4_gemm_quant_out": (_I32, [ctypes.POINTER(_Tensor), ctypes.POINTER(_Tensor), _P, _P, _P, _I64, _P,
+                                            ctypes.POINTER(_Tensor), _P, _SZ, _P, _P]),
             "nvfp4_kv_cache_bytes": (_I64, [_I32, _I32, _I32, _I32, _I32, _I32]),
             "kv_quant_append": (_I32, [ctypes.POINTER(_KVCache), _I32, _I32, _P, _P, _I64, _I64, _P, _SZ, _P, _P]),
             "kv_dequant": (_I32, [ctypes.POINTER(_KVCache), _I32, ctypes.POINTER(_I32), _I32, _P, _P, _P, _P]),
@@ -189,6 +191,26 @@ def nvfp4_gemm(A: QTensor, B: QTensor, bias=None, resid=None, out=None, out_dtyp
     _check("nvfp4_gemm", L.nvfp4_gemm(ctypes.byref(sa), ctypes.byref(sb), _ptr(bias), _ptr(resid), _ptr(out),
                                       out.stride(0), out_dtype, _ptr(status), _stream(stream)))
     return out
+
+
+def nvfp4_gemm_quant_out(A: QTensor, B: QTensor, amax_in, bias=None, resid=None, out=None, q_out=None,
+                         sf_layout=SF_MMA, write_y=True, ws=None, status=None, stream=None):
+    """Y = gA*gB * A . B^T (+bias | +resid) in BF16 and, from the same epilogue, its row-wise NVFP4
+    quantization with the scale of amax_in (a device float).  Returns (Y or None, q_out)."""
+    L = lib()
+    M, N = A.rows, B.rows
+    if out is None and write_y:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=A.codes.device)
+    if q_out is None:
+        q_out = QTensor(M, N, sf_layout, A.codes.device)
+    if ws is None:
+        ws = _ws(L.nvfp4_quantize_workspace(M, N), A.codes.device)
+    ldy = out.stride(0) if out is not None else (resid.stride(0) if resid is not None else N)
+    sa, sb, sq = A.struct(), B.struct(), q_out.struct()
+    _check("nvfp4_gemm_quant_out", L.nvfp4_gemm_quant_out(ctypes.byref(sa), ctypes.byref(sb), _ptr(bias), _ptr(resid),
+                                                          _ptr(out), ldy, _ptr(amax_in), ctypes.byref(sq), _ptr(ws),
+                                                          ws.numel(), _ptr(status), _stream(stream)))
+    return out, q_out
 
 
 class KVCache:

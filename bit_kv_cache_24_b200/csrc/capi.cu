@@ -66,6 +66,44 @@ bool too_large(int64_t rows, int64_t cols) {
     return (uint64_t)(rows + 128) * (uint64_t)(cols + 128) >= (1ull << 35);
 }
 
+// Shared argument checks and GemmArgs of nvfp4_gemm / nvfp4_gemm_quant_out (y may be null only
+// when allow_no_y).
+nvfp4_status gemm_args(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16, const void *resid_bf16,
+                       void *y, int64_t ldy, int32_t y_dtype, bool allow_no_y, int32_t *dev_status, GemmArgs &a) {
+    if (!A || !B || (!y && !allow_no_y) || !A->codes || !B->codes || !A->sf || !B->sf || !A->g || !B->g)
+        return NVFP4_ERR_INVALID_ARG;
+    if (A->rows <= 0 || B->rows <= 0 || A->cols <= 0 || A->cols != B->cols) return NVFP4_ERR_INVALID_ARG;
+    if (bias_bf16 && resid_bf16) return NVFP4_ERR_INVALID_ARG;
+    if (y_dtype != NVFP4_OUT_BF16 && y_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
+    if ((y || resid_bf16) && ldy < B->rows) return NVFP4_ERR_INVALID_ARG;
+    if (A->sf_layout != NVFP4_SF_MMA || B->sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_UNSUPPORTED;
+    if ((B->rows & 7) || ((y || resid_bf16) && (ldy & 7))) return NVFP4_ERR_UNSUPPORTED;
+    if (!aligned16(A->codes) || !aligned16(B->codes) || !aligned16(A->sf) || !aligned16(B->sf) || (y && !aligned16(y)))
+        return NVFP4_ERR_UNSUPPORTED;
+    if ((bias_bf16 && !aligned16(bias_bf16)) || (resid_bf16 && !aligned16(resid_bf16))) return NVFP4_ERR_UNSUPPORTED;
+    if ((A->rows + 127) / 128 > 0x7FFFFFFF / 128) return NVFP4_ERR_UNSUPPORTED;
+    a = GemmArgs{};
+    a.a_codes = A->codes;
+    a.b_codes = B->codes;
+    a.a_sf = A->sf;
+    a.b_sf = B->sf;
+    a.ga = A->g;
+    a.gb = B->g;
+    a.M = A->rows;
+    a.N = B->rows;
+    a.K = A->cols;
+    a.a_pitch = codes_pitch(A->cols);
+    a.b_pitch = codes_pitch(B->cols);
+    a.bias = static_cast<const uint16_t *>(bias_bf16);
+    a.resid = static_cast<const uint16_t *>(resid_bf16);
+    a.y = y;
+    a.ldy = ldy;
+    a.y_f32 = y_dtype == NVFP4_OUT_F32;
+    a.status = dev_status;
+    return NVFP4_OK;
+}
+
+
 bool tensor_ok(const nvfp4_tensor *t, int64_t rows, int64_t cols) {
     return t && t->codes && t->sf && t->g && t->rows == rows && t->cols == cols &&
            (t->sf_layout == NVFP4_SF_LINEAR || t->sf_layout == NVFP4_SF_MMA);
@@ -201,40 +239,46 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
 nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16,
                         const void *resid_bf16, void *y, int64_t ldy, int32_t y_dtype, int32_t *dev_status,
                         nvfp4_stream stream) {
-    if (!A || !B || !y || !A->codes || !B->codes || !A->sf || !B->sf || !A->g || !B->g)
-        return NVFP4_ERR_INVALID_ARG;
-    if (A->rows <= 0 || B->rows <= 0 || A->cols <= 0 || A->cols != B->cols) return NVFP4_ERR_INVALID_ARG;
-    if (bias_bf16 && resid_bf16) return NVFP4_ERR_INVALID_ARG;
-    if (y_dtype != NVFP4_OUT_BF16 && y_dtype != NVFP4_OUT_F32) return NVFP4_ERR_INVALID_ARG;
-    if (ldy < B->rows) return NVFP4_ERR_INVALID_ARG;
-    if (A->sf_layout != NVFP4_SF_MMA || B->sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_UNSUPPORTED;
-    if ((B->rows & 7) || (ldy & 7)) return NVFP4_ERR_UNSUPPORTED;
-    if (!aligned16(A->codes) || !aligned16(B->codes) || !aligned16(A->sf) || !aligned16(B->sf) || !aligned16(y))
-        return NVFP4_ERR_UNSUPPORTED;
-    if ((bias_bf16 && !aligned16(bias_bf16)) || (resid_bf16 && !aligned16(resid_bf16))) return NVFP4_ERR_UNSUPPORTED;
-    if ((A->rows + 127) / 128 > 0x7FFFFFFF / 128) return NVFP4_ERR_UNSUPPORTED;
-    nvfp4_status st = check_device();
+    GemmArgs a;
+    nvfp4_status st = gemm_args(A, B, bias_bf16, resid_bf16, y, ldy, y_dtype, false, dev_status, a);
     if (st != NVFP4_OK) return st;
-    GemmArgs a{};
-    a.a_codes = A->codes;
-    a.b_codes = B->codes;
-    a.a_sf = A->sf;
-    a.b_sf = B->sf;
-    a.ga = A->g;
-    a.gb = B->g;
-    a.M = A->rows;
-    a.N = B->rows;
-    a.K = A->cols;
-    a.a_pitch = codes_pitch(A->cols);
-    a.b_pitch = codes_pitch(B->cols);
-    a.bias = static_cast<const uint16_t *>(bias_bf16);
-    a.resid = static_cast<const uint16_t *>(resid_bf16);
-    a.y = y;
-    a.ldy = ldy;
-    a.y_f32 = y_dtype == NVFP4_OUT_F32;
-    a.status = dev_status;
+    st = check_device();
+    if (st != NVFP4_OK) return st;
     cudaError_t e = launch_gemm(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_gemm");
+}
+
+nvfp4_status nvfp4_gemm_quant_out(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16,
+                                  const void *resid_bf16, void *y_bf16, int64_t ldy, const float *amax_in,
+                                  const nvfp4_tensor *q_out, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                  nvfp4_stream stream) {
+    GemmArgs a;
+    nvfp4_status st = gemm_args(A, B, bias_bf16, resid_bf16, y_bf16, ldy, NVFP4_OUT_BF16, true, dev_status, a);
+    if (st != NVFP4_OK) return st;
+    if (!amax_in || !ws || ws_bytes < kTensorScratchBytes) return NVFP4_ERR_INVALID_ARG;
+    if (!tensor_ok(q_out, A->rows, B->rows)) return NVFP4_ERR_INVALID_ARG;
+    if ((B->rows & 63) || !aligned16(q_out->codes) || !aligned16(q_out->sf) || !aligned16(ws))
+        return NVFP4_ERR_UNSUPPORTED;
+    st = check_device();
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    ScaleRecord *rec = reinterpret_cast<ScaleRecord *>(static_cast<uint8_t *>(ws) + kRecordOffset);
+    RecJobs rj{};
+    rj.njobs = 1;
+    rj.npartial = 0;
+    rj.job[0].partial = nullptr;
+    rj.job[0].amax_in = amax_in;
+    rj.job[0].rec = rec;
+    rj.job[0].g_out[0] = q_out->g;
+    rj.job[0].g_out[1] = nullptr;
+    a.q_rec = rec;
+    a.q_codes = q_out->codes;
+    a.q_sf = q_out->sf;
+    a.q_pitch = codes_pitch(B->rows);
+    a.q_sf_layout = q_out->sf_layout;
+    cudaError_t e = launch_scale_record(rj, dev_status, s);
+    if (e == cudaSuccess) e = launch_gemm(a, s);
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_gemm_quant_out");
 }
 
 int64_t nvfp4_kv_cache_bytes(int32_t layers, int32_t heads, int32_t head_dim, int32_t slots, int32_t slot_tokens,

@@ -28,6 +28,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "launch.h"
 
 namespace nvfp4 {
@@ -188,6 +189,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
     griddep_wait();                                       // operands written by earlier kernels
     griddep_launch_dependents();
+    __shared__ SmemRecord qrec;                           // NVFP4-emitting epilogue only
+    if (args.q_rec) {
+        load_record_plain(args.q_rec, qrec);
+        __syncthreads();
+    }
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -295,6 +301,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
         // ---------------------------------------------------------------- epilogue (warps 2..5)
         const int sub = warp & 3;                         // tensor-memory lane quarter of this warp
         const float alpha = __fmul_rn(*args.ga, *args.gb);
+        const bool quant = args.q_rec && qrec.ok;
+        const int64_t q_rows = args.q_sf_layout ? 128 * ceil_div(M, 128) : M;
         uint32_t acc_phase = 0;
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
             if (!warp_wait(bar_tmem_full, acc_phase)) break;
@@ -308,7 +316,10 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 uint32_t r[32];
                 tc_ld32(trow + c * 32, r);
                 const int64_t n0 = (int64_t)nb * BN + c * 32;
-                if (!row_ok || n0 >= N) continue;
+                if (!row_ok || n0 >= N) {
+                    if (quant && n0 < N && m < q_rows) store_sf_pair(args, m, n0 >> 4, 0u);   // scale padding rows
+                    continue;
+                }
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(alpha, __uint_as_float(r[i]));
@@ -338,13 +349,18 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     }
                 }
                 if (!args.y_f32) {
-                    uint16_t *yrow = reinterpret_cast<uint16_t *>(args.y) + m * args.ldy + n0;
+                    uint32_t w[16];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        if (n0 + 8 * q >= N) break;
-                        stg_v4(yrow + 8 * q, make_uint4(bf16x2(v[8 * q], v[8 * q + 1]), bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                                        bf16x2(v[8 * q + 4], v[8 * q + 5]), bf16x2(v[8 * q + 6], v[8 * q + 7])));
+                    for (int i = 0; i < 16; ++i) w[i] = bf16x2(v[2 * i], v[2 * i + 1]);
+                    if (args.y) {
+                        uint16_t *yrow = reinterpret_cast<uint16_t *>(args.y) + m * args.ldy + n0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            if (n0 + 8 * q >= N) break;
+                            stg_v4(yrow + 8 * q, make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
+                        }
                     }
+                    if (quant) emit_nvfp4_chunk(args, qrec, m, n0, w);
                 } else {
                     float *yrow = reinterpret_cast<float *>(args.y) + m * args.ldy + n0;
 #pragma unroll

@@ -31,6 +31,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "launch.h"
 
 namespace nvfp4 {
@@ -215,6 +216,11 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
     const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
     griddep_wait();                                       // operands written by earlier kernels
     griddep_launch_dependents();
+    __shared__ SmemRecord qrec;                           // NVFP4-emitting epilogue only
+    if (args.q_rec) {
+        load_record_plain(args.q_rec, qrec);
+        __syncthreads();
+    }
 
     auto give_up = [&]() {
         *abort_flag = 1;
@@ -328,6 +334,8 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
         const int half = (warp - EPI_WARP0) >> 2;         // which 128 of the 256 columns
         const uint32_t lead_tmem_empty = map_to_rank(bar_tmem_empty, 0);
         const float alpha = __fmul_rn(*args.ga, *args.gb);
+        const bool quant = args.q_rec && qrec.ok;
+        const int64_t q_rows = args.q_sf_layout ? 128 * ceil_div(M, 128) : M;
         uint32_t acc_phase = 0;
         for (int t = cluster; t < num_tiles; t += nclusters) {
             if (!warp_wait(bar_tmem_full, acc_phase)) break;
@@ -349,7 +357,10 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int64_t n0 = (int64_t)nb * BN + half * 128 + c * 32;
-                if (!row_ok || n0 >= N) continue;
+                if (!row_ok || n0 >= N) {
+                    if (quant && n0 < N && m < q_rows) store_sf_pair(args, m, n0 >> 4, 0u);   // scale padding rows
+                    continue;
+                }
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(alpha, __uint_as_float(r[c][i]));
@@ -368,13 +379,18 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
                     }
                 }
                 if (!args.y_f32) {
-                    uint16_t *yrow = reinterpret_cast<uint16_t *>(args.y) + m * args.ldy + n0;
+                    uint32_t w[16];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        if (n0 + 8 * g >= N) break;
-                        stg_v4(yrow + 8 * g, make_uint4(bf16x2(v[8 * g], v[8 * g + 1]), bf16x2(v[8 * g + 2], v[8 * g + 3]),
-                                                        bf16x2(v[8 * g + 4], v[8 * g + 5]), bf16x2(v[8 * g + 6], v[8 * g + 7])));
+                    for (int i = 0; i < 16; ++i) w[i] = bf16x2(v[2 * i], v[2 * i + 1]);
+                    if (args.y) {
+                        uint16_t *yrow = reinterpret_cast<uint16_t *>(args.y) + m * args.ldy + n0;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (n0 + 8 * g >= N) break;
+                            stg_v4(yrow + 8 * g, make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]));
+                        }
                     }
+                    if (quant) emit_nvfp4_chunk(args, qrec, m, n0, w);
                 } else {
                     float *yrow = reinterpret_cast<float *>(args.y) + m * args.ldy + n0;
 #pragma unroll

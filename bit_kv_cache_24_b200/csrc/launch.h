@@ -110,6 +110,13 @@ struct GemmArgs {
     int64_t ldy;
     int32_t y_f32;
     int32_t *status;
+    // optional NVFP4-emitting epilogue: the row-wise quantization of the BF16 output with the
+    // scale record q_rec (computed from a given amax); y may then be null
+    const ScaleRecord *q_rec;
+    uint8_t *q_codes;
+    uint8_t *q_sf;
+    int64_t q_pitch;
+    int32_t q_sf_layout;
 };
 
 cudaError_t launch_gemm(const GemmArgs &args, cudaStream_t s);

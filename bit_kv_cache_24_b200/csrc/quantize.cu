@@ -96,13 +96,6 @@ __device__ uint32_t reduce_partials(const uint32_t *partial, int n, uint32_t *re
 }
 static_assert(kMaxPartials % kThreads == 0, "partials split evenly over the threads");
 
-// The per-tensor scale record in shared memory, loaded by every quantize CTA.
-struct SmemRecord {
-    float r_tab[128];
-    float den, inv_den;
-    uint32_t ok;
-};
-
 __device__ __forceinline__ uint32_t ldg_cg_u32(const void *p) {
     uint32_t v;
     asm volatile("ld.global.cg.u32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -125,42 +118,6 @@ __device__ __forceinline__ void load_record(const ScaleRecord *rec, SmemRecord &
         s.den = kL2 ? __uint_as_float(ldg_cg_u32(&rec->den)) : rec->den;
         s.inv_den = kL2 ? __uint_as_float(ldg_cg_u32(&rec->inv_den)) : rec->inv_den;
         s.ok = kL2 ? ldg_cg_u32(&rec->ok) : rec->ok;
-    }
-}
-
-// ---- the 16-block step --------------------------------------------------------------------------
-//
-// sf = e4m3(RN(b / den)).  The quotient comes from q0 = RN(b * y), y = RN(1/den), corrected once:
-// q = RN(q0 + RN(b - q0 * den) * y) with both steps fused multiply-adds.  This is the last step of
-// Markstein's division and returns RN(b/den) exactly as long as the residual b - q0*den does not
-// underflow; b >= 2^-100 and den >= 2^-125 (where y is stored nonzero) keep it normal, and every
-// other case takes the IEEE division.  (An exhaustive host-side check over all positive finite
-// BF16 b and ~800 den values, quotients up to 448, found no difference.)  r = 1/d comes from the
-// record's table; d == 0 gives r == 0, meaning every code of the block is +0.
-__device__ __forceinline__ BlockScale block_scale(float b, const SmemRecord &rec) {
-    BlockScale s;
-    float q;
-    if (b >= 0x1p-100f && rec.inv_den != 0.0f) {
-        const float q0 = __fmul_rn(b, rec.inv_den);
-        q = __fmaf_rn(__fmaf_rn(-q0, rec.den, b), rec.inv_den, q0);
-    } else {
-        q = __fdiv_rn(b, rec.den);
-    }
-    s.sf = (b == 0.0f) ? 0u : e4m3(q);
-    s.r = rec.r_tab[s.sf];
-    s.r_inf = isinf(s.r);
-    return s;
-}
-
-__device__ __forceinline__ void quantize16(const uint32_t w[8], const SmemRecord &rec,
-                                           uint32_t &c0, uint32_t &c1, uint32_t &sf) {
-    const uint32_t bm = absmax_bits16(w);
-    const BlockScale s = block_scale(__uint_as_float(bm << 16), rec);
-    sf = s.sf;
-    c0 = c1 = 0;
-    if (s.r != 0.0f) {
-        c0 = encode8(w, s);
-        c1 = encode8(w + 4, s);
     }
 }
 

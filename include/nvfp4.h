@@ -155,6 +155,24 @@ NVFP4_API nvfp4_status nvfp4_gemm(const nvfp4_tensor *A, const nvfp4_tensor *B, 
                         const void *resid_bf16, void *y, int64_t ldy, int32_t y_dtype,
                         int32_t *dev_status, nvfp4_stream stream);
 
+/*
+ * nvfp4_gemm_quant_out -- nvfp4_gemm whose epilogue also emits the row-wise NVFP4 quantization
+ * of its BF16 output Y (the next linear layer's A operand in a W4A4 network), with the
+ * per-tensor scale fixed in advance: g = amax_in / 2688 (amax_in: DEVICE float, e.g. the amax of
+ * the previous step's output; values above it saturate).  q_out (rows = M, cols = N, either
+ * scale layout) receives exactly nvfp4_quantize(Y, NVFP4_ROWWISE, amax_in) of the BF16 Y this
+ * call computes, codes and scales including all padding; q_out->g receives g.  y_bf16 may be
+ * NULL (then only q_out is written; ldy is used for resid_bf16 only).  Requires N % 64 == 0, the
+ * nvfp4_gemm requirements otherwise, and ws of nvfp4_quantize_workspace bytes (the scale record).
+ * A non-finite amax_in sets NVFP4_ERR_NONFINITE in *dev_status and leaves q_out unwritten.
+ * It fuses the activation quantization of the W4A4 path (LongLive-2.0 abstract: NVFP4 linear
+ * layers in training and inference) into the producing GEMM.
+ */
+NVFP4_API nvfp4_status nvfp4_gemm_quant_out(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16,
+                                  const void *resid_bf16, void *y_bf16, int64_t ldy, const float *amax_in,
+                                  const nvfp4_tensor *q_out, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                  nvfp4_stream stream);
+
 /* Bytes of each cache array: which = 0 codes (one of K/V), 1 scales (one of K/V), 2 g (one of
  * K/V); -1 on bad arguments. */
 NVFP4_API int64_t nvfp4_kv_cache_bytes(int32_t layers, int32_t heads, int32_t head_dim, int32_t slots,
