@@ -24,7 +24,7 @@ def _worker(rank, world, port, out):
 
 def test_two_rank_max_and_aggregate():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, 29517, out), nprocs=world, join=True)
     assert out[0] == out[1] == (2.0, 10.0)        # 2 ranks x 10 units / 2.0 s
