@@ -207,8 +207,9 @@ NVFP4_API nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, co
  * No counterpart in the paper: it is a deployment variant of the quantizer above.
  * Same arguments, layouts and results as nvfp4_quantize with amax_in = NULL, bit for bit; the
  * amax partial maxima (1024 slots) and the scale record go to a 5 KB static device array held
- * by every GPU that loads the library.  Nothing is allocated.  A launch needing more than 1024 slots (only possible on
- * GPUs with more than 256 SMs) returns NVFP4_ERR_UNSUPPORTED with a message in
+ * by every GPU that loads the library.  Nothing is allocated.  A launch needing more than 1024
+ * slots (only possible on GPUs with more than 256 SMs) returns NVFP4_ERR_UNSUPPORTED with a
+ * message in
  * nvfp4_last_error().  All calls share the array: calls whose kernels overlap on the GPU race
  * and must be ordered on one stream.  The first call on each device looks up the array's device
  * address; make that first call before any stream capture.
