@@ -103,3 +103,41 @@ def test_full_cache_one_layer(orc):
         qv = orc.Quantized(cv, sv, np.float32(gv), T, row)
         assert np.array_equal(Kh[s], orc.dequant(qk)), s
         assert np.array_equal(Vh[s], orc.dequant(qv)), s
+
+
+def test_full_cache_all_layers(orc):
+    """The whole KV workload geometry: 30 layers x 12 slots of 4680 tokens (24 heads x 128, ~5.8 GB
+    of NVFP4 cache; offsets of the last layers pass 2^31 bytes).  Every slot of every layer is
+    appended; layers 0, 13 and 29 hold their own chunks (the others reuse a few), their slots 0
+    and 11 are compared byte for byte with the oracle's quantizer, and layer 29's full window
+    restore with the oracle's dequantizer of the cache bytes."""
+    H, D, S, T, L = synth.HEADS, synth.HEAD_DIM, synth.KV_APPENDS, synth.CHUNK_TOKENS, 30
+    row = H * D
+    cache = nv.KVCache(L, H, D, S, T)
+    checked = (0, 13, 29)
+    pool = [tuple(t.cuda() for t in synth.kv_chunk(3, s)) for s in range(3)]
+    kept = {}
+    for layer in range(L):
+        for s in range(S):
+            if layer in checked:
+                k, v = synth.kv_chunk(layer, s)
+                if s in (0, S - 1):
+                    kept[(layer, s)] = (k, v)
+                nv.kv_quant_append(cache, layer, s, k.cuda(), v.cuda())
+            else:
+                k, v = pool[(layer + s) % 3]
+                nv.kv_quant_append(cache, layer, s, k, v)
+    K, V = nv.kv_dequant(cache, L - 1, list(range(S)))
+    torch.cuda.synchronize()
+    for (layer, s), (k, v) in kept.items():
+        ck, sk, gk, cv, sv, gv = _slot_bytes(cache, layer, s)
+        _, qk = orc.quantize(k.reshape(T, row))
+        _, qv = orc.quantize(v.reshape(T, row))
+        assert np.array_equal(ck, qk.codes) and np.array_equal(sk, qk.sf) and gk == float(qk.g), (layer, s)
+        assert np.array_equal(cv, qv.codes) and np.array_equal(sv, qv.sf) and gv == float(qv.g), (layer, s)
+    Kh = K.view(torch.int16).cpu().numpy().view(np.uint16).reshape(S, T, row)
+    Vh = V.view(torch.int16).cpu().numpy().view(np.uint16).reshape(S, T, row)
+    for s in range(S):
+        ck, sk, gk, cv, sv, gv = _slot_bytes(cache, L - 1, s)
+        assert np.array_equal(Kh[s], orc.dequant(orc.Quantized(ck, sk, np.float32(gk), T, row))), s
+        assert np.array_equal(Vh[s], orc.dequant(orc.Quantized(cv, sv, np.float32(gv), T, row))), s
