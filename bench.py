@@ -270,6 +270,18 @@ class QKVStep:
         }
 
 
+def workload_config(world):
+    """The workload both arms report (the reference arm times a bounded row sample of it, stated in
+    its cpu_baseline.sample)."""
+    return {"workload": "qkv_chunk_step: A[4680x3072] x W[9216x3072]^T + bias, KV append 4680 tok, "
+                        "KV window 12x4680 tok x 24 heads x 128",
+            "global_batch": M_TOK * world, "seq_len": SLOTS * M_TOK, "parallelism": f"replicas x{world}",
+            "l2": "inputs rotate over 3 sets (~300 MB) and each step streams ~1.1 GB (> 126 MB L2)",
+            "value_def": "GEMM FLOPs per step / time per step (all 5 ops; W and A quantization concurrent), "
+                         "summed over replicas; device time for the GPU arm, host time of the row "
+                         "sample for the reference arm"}
+
+
 def run_ours(args, rank, local_rank, world):
     dist = init_dist(world, "nccl")
     torch.cuda.set_device(local_rank)
@@ -404,11 +416,7 @@ def run_ours(args, rank, local_rank, world):
         "warmup": args.warmup, "ms_per_step": round(max_s * 1e3 / K, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3/16) -> fp32 acc -> bf16",
         "data": "synthetic (seeded; QKV-projection shapes of a 5B video DiT, random-init weights)",
-        "config": {"workload": "qkv_chunk_step: A[4680x3072] x W[9216x3072]^T + bias, KV append 4680 tok, "
-                               "KV window 12x4680 tok x 24 heads x 128",
-                   "global_batch": M_TOK * world, "seq_len": SLOTS * M_TOK, "parallelism": f"replicas x{world}",
-                   "l2": "inputs rotate over 3 sets (~300 MB) and each step streams ~1.1 GB (> 126 MB L2)",
-                   "value_def": "GEMM FLOPs per step / device time per step (all 5 ops; W and A quantization concurrent), summed over replicas"},
+        "config": workload_config(world),
         "gpu_launches": launches,
         "kernels": kernels, "roofline": roofline, "clocks": clk, "e2e": e2e,
         "device_status": status,
@@ -493,8 +501,7 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)",
             "data": "synthetic (seeded; same generator as the GPU arm)",
-            "config": {"workload": "qkv_chunk_step (CPU oracle on a row sample)", "global_batch": rows,
-                       "seq_len": SLOTS * rows, "parallelism": "cpu"},
+            "config": workload_config(world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(os.cpu_count(), rows), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
