@@ -1,7 +1,9 @@
 // capi.cu -- the C ABI declared in include/nvfp4.h: argument validation, layout arithmetic,
 // architecture checks and kernel dispatch.  No allocation, no synchronisation.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -18,25 +20,30 @@ nvfp4_status cuda_fail(cudaError_t e, const char *where) {
 }
 
 struct DevInfo {
-    bool probed = false;
+    std::atomic<bool> probed{false};   // set (release) after the fields below
     bool sm100 = false;
     int sms = 148;
 };
 DevInfo g_dev[64];
+std::mutex g_dev_mutex;
 
+// The current device's properties, probed once per device (thread-safe).
 const DevInfo *device_info() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     DevInfo &d = g_dev[dev];
-    if (!d.probed) {
-        int major = 0, minor = 0, sms = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return nullptr;
-        d.sm100 = (major == 10 && minor == 0);
-        d.sms = sms;
-        d.probed = true;
+    if (!d.probed.load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        if (!d.probed.load(std::memory_order_relaxed)) {
+            int major = 0, minor = 0, sms = 0;
+            if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return nullptr;
+            d.sm100 = (major == 10 && minor == 0);
+            d.sms = sms;
+            d.probed.store(true, std::memory_order_release);
+        }
     }
     return &d;
 }

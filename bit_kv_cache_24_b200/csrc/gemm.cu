@@ -24,6 +24,7 @@
 //   - Every mbarrier wait is bounded (2 s); a wait that gives up raises an abort flag shared by
 //     all roles, writes NVFP4_ERR_TIMEOUT to the status word, drains the copies and MMAs this
 //     CTA has in flight (bounded), frees tensor memory and returns.
+#include <atomic>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -415,14 +416,14 @@ bool make_code_map(CUtensorMap *map, const void *ptr, int64_t rows, int64_t pitc
 
 cudaError_t launch_gemm(const GemmArgs &args, cudaStream_t s) {
     if (args.M > BM) return launch_gemm_2sm(args, s);     // CTA pairs once M spans two row blocks
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];             // per device; a repeated set is harmless
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(nvfp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     CUtensorMap ma, mb;
     if (!make_code_map(&ma, args.a_codes, args.M, args.a_pitch, BM) ||

@@ -27,6 +27,7 @@
 // Scale tiles are read through 2-D tensor maps over the 512-byte atoms (viewed as uint64), so
 // atom rows past M or N are zero-filled by TMA like the code tiles.
 // Every wait is time-bounded; a wait that gives up reports NVFP4_ERR_TIMEOUT and the CTA returns.
+#include <atomic>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -442,14 +443,14 @@ bool encode_2d(CUtensorMap *map, CUtensorMapDataType dt, uint32_t esize, const v
 }  // namespace
 
 cudaError_t launch_gemm_2sm(const GemmArgs &args, cudaStream_t s) {
-    static bool attr_set[64] = {false};
+    static std::atomic<bool> attr_set[64];             // per device; a repeated set is harmless
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(nvfp4_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
         if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     const int64_t ksteps = ceil_div(args.K, KSTEP);        // scale atoms per 128-row block
     Maps maps;
