@@ -78,8 +78,13 @@ def lib():
             "nvfp4_gemm": (_I32, [ctypes.POINTER(_Tensor), ctypes.POINTER(_Tensor), _P, _P, _P, _I64, _I32, _P, _P]),
             "nvfp4_gemm_quant_out": (_I32, [ctypes.POINTER(_Tensor), ctypes.POINTER(_Tensor), _P, _P, _P, _I64, _P,
                                             ctypes.POINTER(_Tensor), _P, _SZ, _P, _P]),
+            "nvfp4_gemm_colamax_workspace": (_SZ, [_I64, _I64]),
+            "nvfp4_gemm_colamax": (_I32, [ctypes.POINTER(_Tensor), ctypes.POINTER(_Tensor), _P, _P, _P, _I64, _I64, _P,
+                                          _P, _SZ, _P, _P]),
             "nvfp4_kv_cache_bytes": (_I64, [_I32, _I32, _I32, _I32, _I32, _I32]),
             "kv_quant_append": (_I32, [ctypes.POINTER(_KVCache), _I32, _I32, _P, _P, _I64, _I64, _P, _SZ, _P, _P]),
+            "kv_quant_append_amax": (_I32, [ctypes.POINTER(_KVCache), _I32, _I32, _P, _P, _I64, _I64, _P, _P, _SZ, _P,
+                                            _P]),
             "kv_dequant": (_I32, [ctypes.POINTER(_KVCache), _I32, ctypes.POINTER(_I32), _I32, _P, _P, _P, _P]),
             "nvfp4_encode_elements": (_I32, [_P, _I64, _P, _P, _P]),
             "nvfp4_selftest_wait_timeout": (_I32, [_P, _I64, _P]),
@@ -213,6 +218,26 @@ def nvfp4_gemm_quant_out(A: QTensor, B: QTensor, amax_in, bias=None, resid=None,
     return out, q_out
 
 
+def nvfp4_gemm_colamax(A: QTensor, B: QTensor, group_cols, bias=None, resid=None, out=None, amax_out=None,
+                       ws=None, status=None, stream=None):
+    """Y = gA*gB * A . B^T (+bias | +resid) in BF16 and max |Y| per group of group_cols columns
+    (reduced in the epilogue).  Returns (Y, amax_out [N / group_cols] float32 on the device)."""
+    L = lib()
+    M, N = A.rows, B.rows
+    dev = A.codes.device
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    if amax_out is None:
+        amax_out = torch.empty(N // group_cols, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _ws(L.nvfp4_gemm_colamax_workspace(M, N), dev)
+    sa, sb = A.struct(), B.struct()
+    _check("nvfp4_gemm_colamax", L.nvfp4_gemm_colamax(ctypes.byref(sa), ctypes.byref(sb), _ptr(bias), _ptr(resid),
+                                                      _ptr(out), out.stride(0), group_cols, _ptr(amax_out), _ptr(ws),
+                                                      ws.numel(), _ptr(status), _stream(stream)))
+    return out, amax_out
+
+
 class KVCache:
     """Caller-owned chunk-slot NVFP4 KV cache storage (device arrays + host slot lengths)."""
 
@@ -242,9 +267,10 @@ class KVCache:
         return self.len[layer * self.slots + slot]
 
 
-def kv_quant_append(cache: KVCache, layer, slot, k, v, status=None, stream=None):
+def kv_quant_append(cache: KVCache, layer, slot, k, v, status=None, stream=None, amax_kv=None):
     """Quantize one chunk's K and V ([ntok, heads, head_dim] or [ntok, heads*head_dim] BF16, rows
-    possibly strided) into slot `slot` of `layer` in place."""
+    possibly strided) into slot `slot` of `layer` in place.  amax_kv: optional device float[2]
+    (amax of K, of V), e.g. from nvfp4_gemm_colamax; then no amax pass runs."""
     row = cache.heads * cache.head_dim
     k2 = k.reshape(k.shape[0], row) if k.dim() == 3 else k
     v2 = v.reshape(v.shape[0], row) if v.dim() == 3 else v
@@ -252,9 +278,15 @@ def kv_quant_append(cache: KVCache, layer, slot, k, v, status=None, stream=None)
     _bf16_2d(v2, "v")
     if k2.stride(0) != v2.stride(0) or k2.shape != v2.shape:
         raise ValueError("k and v must have the same shape and row stride")
-    _check("kv_quant_append", lib().kv_quant_append(ctypes.byref(cache._c), layer, slot, _ptr(k2), _ptr(v2),
-                                                    k2.shape[0], k2.stride(0), _ptr(cache.ws), cache.ws.numel(),
-                                                    _ptr(status), _stream(stream)))
+    if amax_kv is None:
+        _check("kv_quant_append", lib().kv_quant_append(ctypes.byref(cache._c), layer, slot, _ptr(k2), _ptr(v2),
+                                                        k2.shape[0], k2.stride(0), _ptr(cache.ws), cache.ws.numel(),
+                                                        _ptr(status), _stream(stream)))
+    else:
+        _check("kv_quant_append_amax", lib().kv_quant_append_amax(ctypes.byref(cache._c), layer, slot, _ptr(k2),
+                                                                  _ptr(v2), k2.shape[0], k2.stride(0), _ptr(amax_kv),
+                                                                  _ptr(cache.ws), cache.ws.numel(), _ptr(status),
+                                                                  _stream(stream)))
 
 
 def kv_dequant(cache: KVCache, layer, slots, k_out=None, v_out=None, status=None, stream=None):

@@ -288,6 +288,34 @@ nvfp4_status nvfp4_gemm_quant_out(const nvfp4_tensor *A, const nvfp4_tensor *B, 
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_gemm_quant_out");
 }
 
+size_t nvfp4_gemm_colamax_workspace(int64_t M, int64_t N) {
+    if (M <= 0 || N <= 0) return 0;
+    return (size_t)ceil_div(M, 32) * (size_t)ceil_div(N, 128) * sizeof(uint32_t);
+}
+
+nvfp4_status nvfp4_gemm_colamax(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16,
+                                const void *resid_bf16, void *y_bf16, int64_t ldy, int64_t group_cols,
+                                float *amax_out, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                nvfp4_stream stream) {
+    GemmArgs a;
+    nvfp4_status st = gemm_args(A, B, bias_bf16, resid_bf16, y_bf16, ldy, NVFP4_OUT_BF16, false, dev_status, a);
+    if (st != NVFP4_OK) return st;
+    const int64_t M = A->rows, N = B->rows;
+    if (!amax_out || !ws || group_cols <= 0 || ws_bytes < nvfp4_gemm_colamax_workspace(M, N))
+        return NVFP4_ERR_INVALID_ARG;
+    if ((group_cols & 255) || N % group_cols || !aligned16(ws)) return NVFP4_ERR_UNSUPPORTED;
+    st = check_device();
+    if (st != NVFP4_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    a.cam_partial = static_cast<uint32_t *>(ws);
+    a.cam_n128 = N / 128;
+    cudaError_t e = launch_gemm(a, s);
+    if (e == cudaSuccess)
+        e = launch_colamax_finish(a.cam_partial, ceil_div(M, 32), N / 128, group_cols, N / group_cols, amax_out,
+                                  dev_status, s);
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_gemm_colamax");
+}
+
 int64_t nvfp4_kv_cache_bytes(int32_t layers, int32_t heads, int32_t head_dim, int32_t slots, int32_t slot_tokens,
                              int32_t which) {
     if (layers <= 0 || heads <= 0 || head_dim <= 0 || slots <= 0 || slot_tokens <= 0) return -1;
@@ -309,6 +337,13 @@ static bool kv_ok(const nvfp4_kv_cache *c) {
 nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int32_t slot, const void *k_bf16,
                              const void *v_bf16, int64_t ntok, int64_t ld, void *ws, size_t ws_bytes,
                              int32_t *dev_status, nvfp4_stream stream) {
+    return kv_quant_append_amax(cache, layer, slot, k_bf16, v_bf16, ntok, ld, nullptr, ws, ws_bytes, dev_status,
+                                stream);
+}
+
+nvfp4_status kv_quant_append_amax(nvfp4_kv_cache *cache, int32_t layer, int32_t slot, const void *k_bf16,
+                                  const void *v_bf16, int64_t ntok, int64_t ld, const float *amax_kv, void *ws,
+                                  size_t ws_bytes, int32_t *dev_status, nvfp4_stream stream) {
     if (!kv_ok(cache) || !k_bf16 || !v_bf16 || !ws) return NVFP4_ERR_INVALID_ARG;
     if (layer < 0 || layer >= cache->layers || slot < 0 || slot >= cache->slots) return NVFP4_ERR_INVALID_ARG;
     const int64_t row = (int64_t)cache->heads * cache->head_dim;
@@ -343,12 +378,12 @@ nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int32_t slot,
         j.partial = reinterpret_cast<uint32_t *>(scratch);
         j.rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
         rj.job[i].partial = j.partial;
-        rj.job[i].amax_in = nullptr;
+        rj.job[i].amax_in = amax_kv ? amax_kv + i : nullptr;
         rj.job[i].rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
         rj.job[i].g_out[0] = (i == 0 ? cache->g_k : cache->g_v) + slot_index;
         rj.job[i].g_out[1] = nullptr;
     }
-    cudaError_t e = launch_amax(jobs, dev_status, nullptr, s);
+    cudaError_t e = amax_kv ? cudaSuccess : launch_amax(jobs, dev_status, nullptr, s);
     if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
     if (e == cudaSuccess) e = launch_quantize_rows(jobs, s);
     if (e != cudaSuccess) return cuda_fail(e, "kv_quant_append");

@@ -312,6 +312,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
             const int64_t m = (int64_t)mb * BM + sub * 32 + lane;
             const bool row_ok = m < M;
             const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16) + ACC_COL;
+            uint32_t cam0 = 0, cam1 = 0;                  // max |Y| of this warp's two 32 x 128 blocks
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
@@ -362,6 +363,11 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                         }
                     }
                     if (quant) emit_nvfp4_chunk(args, qrec, m, n0, w);
+                    if (args.cam_partial) {
+                        const uint32_t b = max(absmax_bits16(w), absmax_bits16(w + 8));
+                        if (c < 4) cam0 = max(cam0, b);
+                        else cam1 = max(cam1, b);
+                    }
                 } else {
                     float *yrow = reinterpret_cast<float *>(args.y) + m * args.ldy + n0;
 #pragma unroll
@@ -370,6 +376,19 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                         stg_v4(yrow + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
                                                         __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
                     }
+                }
+            }
+            if (args.cam_partial) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    cam0 = max(cam0, __shfl_xor_sync(0xFFFFFFFFu, cam0, o));
+                    cam1 = max(cam1, __shfl_xor_sync(0xFFFFFFFFu, cam1, o));
+                }
+                const int64_t r32 = ((int64_t)mb * BM + sub * 32) >> 5;
+                const int64_t c128 = ((int64_t)nb * BN) >> 7;
+                if (lane == 0 && r32 < ceil_div(M, 32)) {
+                    if (c128 < args.cam_n128) args.cam_partial[r32 * args.cam_n128 + c128] = cam0;
+                    if (c128 + 1 < args.cam_n128) args.cam_partial[r32 * args.cam_n128 + c128 + 1] = cam1;
                 }
             }
             tc_fence_before();

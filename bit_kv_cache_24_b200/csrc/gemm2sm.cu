@@ -355,6 +355,7 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
             __syncwarp();
             if (lane == 0)
                 asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" :: "r"(lead_tmem_empty) : "memory");
+            uint32_t cam = 0;                             // max |Y| of this warp's 32 x 128 block
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int64_t n0 = (int64_t)nb * BN + half * 128 + c * 32;
@@ -392,6 +393,7 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
                         }
                     }
                     if (quant) emit_nvfp4_chunk(args, qrec, m, n0, w);
+                    if (args.cam_partial) cam = max(cam, max(absmax_bits16(w), absmax_bits16(w + 8)));
                 } else {
                     float *yrow = reinterpret_cast<float *>(args.y) + m * args.ldy + n0;
 #pragma unroll
@@ -401,6 +403,14 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
                                                         __float_as_uint(v[4 * g + 2]), __float_as_uint(v[4 * g + 3])));
                     }
                 }
+            }
+            if (args.cam_partial) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) cam = max(cam, __shfl_xor_sync(0xFFFFFFFFu, cam, o));
+                const int64_t r32 = ((int64_t)mb * BM + (int64_t)rank * BM_CTA + q * 32) >> 5;
+                const int64_t c128 = ((int64_t)nb * BN + half * 128) >> 7;
+                if (lane == 0 && r32 < ceil_div(M, 32) && c128 < args.cam_n128)
+                    args.cam_partial[r32 * args.cam_n128 + c128] = cam;
             }
             acc_phase ^= 1;
         }

@@ -117,7 +117,16 @@ struct GemmArgs {
     uint8_t *q_sf;
     int64_t q_pitch;
     int32_t q_sf_layout;
+    // optional per-block amax of the BF16 output: max |Y| (BF16 magnitude bits) of each 32-row x
+    // 128-column block, at cam_partial[(row / 32) * cam_n128 + col / 128] (N % 256 == 0)
+    uint32_t *cam_partial;
+    int64_t cam_n128;
 };
+
+// Column-group amax from the GEMM's block partials: amax_out[g] = max over the blocks of columns
+// [g * group_cols, (g + 1) * group_cols) (one CTA per group).
+cudaError_t launch_colamax_finish(const uint32_t *partial, int64_t rows32, int64_t n128, int64_t group_cols,
+                                  int64_t groups, float *amax_out, int32_t *status, cudaStream_t s);
 
 cudaError_t launch_gemm(const GemmArgs &args, cudaStream_t s);
 // CTA-pair (cta_group::2) variant for M > 128; launch_gemm dispatches to it.

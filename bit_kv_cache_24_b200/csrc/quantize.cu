@@ -184,6 +184,36 @@ __global__ void __launch_bounds__(kThreads) amax_finish_kernel(const uint32_t *p
     }
 }
 
+// Column-group amax of a GEMM output from its per-block partials (nvfp4_gemm_colamax): CTA g
+// reduces the blocks of columns [g * group_cols, (g + 1) * group_cols); inf/NaN reports
+// NVFP4_ERR_NONFINITE and stores NaN.
+__global__ void __launch_bounds__(kThreads) colamax_finish_kernel(const uint32_t *partial, int64_t rows32, int64_t n128,
+                                                                  int64_t group_cols, float *amax_out, int32_t *status) {
+    griddep_wait();
+    griddep_launch_dependents();
+    __shared__ uint32_t red[kWarps];
+    const int64_t cpg = group_cols >> 7, c0 = (int64_t)blockIdx.x * cpg;
+    const int64_t n = rows32 * cpg;
+    uint32_t m = 0;
+    for (int64_t i = threadIdx.x; i < n; i += kThreads) {
+        const int64_t r = i / cpg;
+        m = max(m, partial[r * n128 + c0 + (i - r * cpg)]);
+    }
+    m = warp_max(m);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t b = 0;
+        for (int w = 0; w < kWarps; ++w) b = max(b, red[w]);
+        if (b >= 0x7F80u) {
+            set_status(status, NVFP4_ERR_NONFINITE);
+            amax_out[blockIdx.x] = __uint_as_float(0x7FC00000u);
+        } else {
+            amax_out[blockIdx.x] = __uint_as_float(b << 16);
+        }
+    }
+}
+
 // Pass 2: the scale record of each tensor (one CTA per job) from its partials or its amax_in.
 __global__ void __launch_bounds__(kThreads) scale_record_kernel(const __grid_constant__ RecJobs jobs, int32_t *status) {
     griddep_wait();
@@ -423,6 +453,12 @@ cudaError_t launch_amax(const RowJobs &jobs, int32_t *status, float *amax_out, c
         e = launch_pdl(amax_finish_kernel, dim3(1), dim3(kThreads), 0, s,
                        (const uint32_t *)jobs.job[0].partial, (int)jobs.npartial, amax_out, status);
     return e;
+}
+
+cudaError_t launch_colamax_finish(const uint32_t *partial, int64_t rows32, int64_t n128, int64_t group_cols,
+                                  int64_t groups, float *amax_out, int32_t *status, cudaStream_t s) {
+    return launch_pdl(colamax_finish_kernel, dim3((unsigned)groups), dim3(kThreads), 0, s, partial, rows32, n128,
+                      group_cols, amax_out, status);
 }
 
 cudaError_t launch_scale_record(const RecJobs &jobs, int32_t *status, cudaStream_t s) {

@@ -173,6 +173,20 @@ NVFP4_API nvfp4_status nvfp4_gemm_quant_out(const nvfp4_tensor *A, const nvfp4_t
                                   const nvfp4_tensor *q_out, void *ws, size_t ws_bytes, int32_t *dev_status,
                                   nvfp4_stream stream);
 
+/*
+ * nvfp4_gemm_colamax -- nvfp4_gemm (BF16 output) whose epilogue also reduces max |Y| of the BF16
+ * output over column groups of group_cols columns: amax_out[g] (DEVICE float[N / group_cols]) =
+ * max |Y[:, g*group_cols : (g+1)*group_cols]|, exact (a max of the stored BF16 values), e.g. the
+ * amax of the K and V slices of a fused QKV projection.  Requires group_cols % 256 == 0,
+ * N % group_cols == 0, and ws of nvfp4_gemm_colamax_workspace(M, N) bytes (per-block partial
+ * maxima; no initialisation needed).  inf/NaN in a group sets NVFP4_ERR_NONFINITE and stores NaN.
+ */
+NVFP4_API size_t nvfp4_gemm_colamax_workspace(int64_t M, int64_t N);
+NVFP4_API nvfp4_status nvfp4_gemm_colamax(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16,
+                                const void *resid_bf16, void *y_bf16, int64_t ldy, int64_t group_cols,
+                                float *amax_out, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                nvfp4_stream stream);
+
 /* Bytes of each cache array: which = 0 codes (one of K/V), 1 scales (one of K/V), 2 g (one of
  * K/V); -1 on bad arguments. */
 NVFP4_API int64_t nvfp4_kv_cache_bytes(int32_t layers, int32_t heads, int32_t head_dim, int32_t slots,
@@ -190,6 +204,17 @@ NVFP4_API nvfp4_status kv_quant_append(nvfp4_kv_cache *cache, int32_t layer, int
                              const void *k_bf16, const void *v_bf16, int64_t ntok, int64_t ld,
                              void *ws, size_t ws_bytes, int32_t *dev_status,
                              nvfp4_stream stream);
+
+/*
+ * kv_quant_append_amax -- kv_quant_append with the amax of K and of V given (amax_kv: DEVICE
+ * float[2], K then V; e.g. from nvfp4_gemm_colamax of the GEMM that produced them), so no amax
+ * pass reads K and V.  With the exact amax of the chunk the cache bytes equal kv_quant_append's.
+ * A non-finite amax sets NVFP4_ERR_NONFINITE in *dev_status and leaves the slot unwritten.
+ */
+NVFP4_API nvfp4_status kv_quant_append_amax(nvfp4_kv_cache *cache, int32_t layer, int32_t slot,
+                                  const void *k_bf16, const void *v_bf16, int64_t ntok, int64_t ld,
+                                  const float *amax_kv, void *ws, size_t ws_bytes, int32_t *dev_status,
+                                  nvfp4_stream stream);
 
 /*
  * kv_dequant -- parallel restore of a window of slots of one layer to BF16: the listed slots

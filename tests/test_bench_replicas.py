@@ -38,3 +38,19 @@ def test_single_rank_is_identity():
 def test_arg_defaults_fit_the_contract():
     a = bench.parse_args([])
     assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1 and a.impl == "ours"
+
+
+def test_op_summary_excludes_the_side_stream_op():
+    # event times (ms over K=10 steps) shaped like the QKV step: the side-stream op's time is the
+    # largest but it overlaps the others, so it has no share and is not the dominant op
+    per_op = {"w": 1.6, "a": 0.4, "gemm": 1.0, "kv": 0.2, "deq": 1.4}
+    work = {"w": ("hbm", 1e8), "a": ("hbm", 5e7), "gemm": ("tensor", 2.65e11), "kv": ("hbm", 7e7),
+            "deq": ("hbm", 8.8e8)}
+    k, dom = bench.summarize_ops(per_op, 10, work, {"w"}, 6500.0, 5500.0)
+    assert dom == "deq"
+    assert k["w"]["share"] is None and "side" in k["w"]["stream"]
+    assert abs(sum(v["share"] for v in k.values() if v["share"] is not None) - 1.0) < 1e-3
+    assert k["deq"]["share"] == round(1.4 / 3.0, 4)
+    # 8.8e8 B in 0.14 ms = 6285.7 GB/s; 2.65e11 FLOP in 0.1 ms = 2650 TFLOP/s
+    assert k["deq"]["us_per_launch"] == 140.0 and abs(k["deq"]["achieved"] - 6285.7) < 0.1
+    assert k["gemm"]["unit"] == "TFLOP/s" and abs(k["gemm"]["frac"] - 2650 / 5500) < 1e-4
