@@ -192,12 +192,24 @@ __global__ void __launch_bounds__(kThreads) colamax_finish_kernel(const uint32_t
     griddep_wait();
     griddep_launch_dependents();
     __shared__ uint32_t red[kWarps];
-    const int64_t cpg = group_cols >> 7, c0 = (int64_t)blockIdx.x * cpg;
-    const int64_t n = rows32 * cpg;
+    constexpr int kRowsInFlight = 8;
+    const int64_t cpg = group_cols >> 7;
+    const uint32_t *p = partial + (int64_t)blockIdx.x * cpg;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // lanes walk the group's column blocks, warps its 32-row blocks, eight independent loads in
+    // flight per lane (the partials are few: latency, not bandwidth, sets this kernel's time)
     uint32_t m = 0;
-    for (int64_t i = threadIdx.x; i < n; i += kThreads) {
-        const int64_t r = i / cpg;
-        m = max(m, partial[r * n128 + c0 + (i - r * cpg)]);
+    for (int64_t c = lane; c < cpg; c += 32) {
+        for (int64_t r0 = warp; r0 < rows32; r0 += (int64_t)kWarps * kRowsInFlight) {
+            uint32_t v[kRowsInFlight];
+#pragma unroll
+            for (int u = 0; u < kRowsInFlight; ++u) {
+                const int64_t r = r0 + (int64_t)u * kWarps;
+                v[u] = r < rows32 ? p[r * n128 + c] : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kRowsInFlight; ++u) m = max(m, v[u]);
+        }
     }
     m = warp_max(m);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
