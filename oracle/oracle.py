@@ -280,3 +280,41 @@ class KVCacheModel:
             vs.append(dequant(qv))
         shape = (-1, self.heads, self.head_dim)
         return np.concatenate(ks).reshape(shape), np.concatenate(vs).reshape(shape)
+
+    def attention(self, layer, slots, q, scale, rows=None):
+        """Attention of the queries q over the window of the listed slots: attention() over the
+        BF16 K and V the window restores to."""
+        k, v = self.dequant(layer, slots)
+        return attention(q, k, v, scale, rows=rows)
+
+
+# ---- attention over the restored KV window ---------------------------------------------------
+
+def attention(q, k, v, scale, rows=None):
+    """fp64 softmax attention over a restored KV window (LongLive-2.0 keeps the KV cache in NVFP4
+    and restores it for attention: d9249.github.io review, section "핵심 아이디어 / 구조 / 동작
+    방식"; arXiv abstract on fugumt.com).  For every head h and query row i:
+
+        w_j      = exp(scale * <q[i, h, :], k[j, h, :]>)    over the window's tokens j
+        O[i,h,:] = sum_j w_j v[j, h, :] / sum_j w_j
+
+    q [Tq, H, D], k and v [Tk, H, D]: BF16 (torch CPU tensors or uint16 bit arrays), k and v as the
+    window restores to (KVCacheModel.dequant); scale: the FP32 softmax scale (taken at its FP32
+    value).  No mask: every query attends to every token of the window.  ``rows`` selects query
+    rows (default all).  Returns fp64 [len(rows), H, D].  The per-row maximum of the exponent is
+    subtracted before exp to keep it in range; it cancels in the ratio."""
+    qf = bf16_bits_to_f32(as_u16(q)).astype(np.float64)
+    kf = bf16_bits_to_f32(as_u16(k)).astype(np.float64)
+    vf = bf16_bits_to_f32(as_u16(v)).astype(np.float64)
+    if rows is not None:
+        qf = qf[np.asarray(rows, dtype=np.int64)]
+    tq, heads, d = qf.shape
+    assert kf.shape[1:] == (heads, d) and vf.shape == kf.shape and kf.shape[0] > 0
+    c = np.float64(np.float32(scale))
+    out = np.empty((tq, heads, d), dtype=np.float64)
+    for h in range(heads):
+        e = (qf[:, h, :] @ kf[:, h, :].T) * c              # [tq, Tk] exponents
+        e -= e.max(axis=1, keepdims=True)
+        w = np.exp(e)
+        out[:, h, :] = (w @ vf[:, h, :]) / w.sum(axis=1, keepdims=True)
+    return out
