@@ -10,6 +10,7 @@ Entry points (same names as the C ABI):
   nvfp4_gemm(A, B, bias=None, resid=None, ...) -> BF16 (or FP32) [M, N]
   kv_quant_append(cache, layer, slot, k, v)   in place into a KVCache
   kv_dequant(cache, layer, slots)             -> (K, V) BF16 [tokens, heads, head_dim]
+  kv_attention(cache, layer, slots, q, scale) -> O BF16 [tq, heads, head_dim] (restore fused)
 """
 from __future__ import annotations
 
@@ -86,6 +87,8 @@ def lib():
             "kv_quant_append_amax": (_I32, [ctypes.POINTER(_KVCache), _I32, _I32, _P, _P, _I64, _I64, _P, _P, _SZ, _P,
                                             _P]),
             "kv_dequant": (_I32, [ctypes.POINTER(_KVCache), _I32, ctypes.POINTER(_I32), _I32, _P, _P, _P, _P]),
+            "kv_attention": (_I32, [ctypes.POINTER(_KVCache), _I32, ctypes.POINTER(_I32), _I32, _P, _I64, _I64,
+                                    ctypes.c_float, _P, _I64, _P, _P]),
             "nvfp4_encode_elements": (_I32, [_P, _I64, _P, _P, _P]),
             "nvfp4_selftest_wait_timeout": (_I32, [_P, _I64, _P]),
         }
@@ -301,6 +304,34 @@ def kv_dequant(cache: KVCache, layer, slots, k_out=None, v_out=None, status=None
     _check("kv_dequant", lib().kv_dequant(ctypes.byref(cache._c), layer, arr, len(slots), _ptr(k_out), _ptr(v_out),
                                           _ptr(status), _stream(stream)))
     return k_out, v_out
+
+
+def kv_attention(cache: KVCache, layer, slots, q, scale, out=None, status=None, stream=None):
+    """Softmax attention of q over the listed slots of `layer`, the restore fused into the kernel.
+
+    q: BF16 CUDA tensor [tq, heads, head_dim], or a 2-D [tq, >= heads * head_dim] view with unit
+    column stride (e.g. the Q columns of a fused QKV output). Returns O, BF16 [tq, heads, head_dim]
+    (or `out`, with the same shape rules)."""
+    def rows(t, name):
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == torch.bfloat16):
+            raise TypeError(f"{name} must be a bfloat16 CUDA tensor")
+        if t.dim() == 3 and tuple(t.shape[1:]) == (cache.heads, cache.head_dim) and \
+                t.stride(2) == 1 and t.stride(1) == cache.head_dim:
+            return t.shape[0], t.stride(0)
+        if t.dim() == 2 and t.shape[1] == cache.heads * cache.head_dim and t.stride(1) == 1:
+            return t.shape[0], t.stride(0)
+        raise ValueError(f"{name} must be [tq, heads, head_dim] with contiguous rows")
+    tq, ldq = rows(q, "q")
+    if out is None:
+        out = torch.empty(tq, cache.heads, cache.head_dim, dtype=torch.bfloat16, device=q.device)
+    to, ldo = rows(out, "out")
+    if to != tq:
+        raise ValueError("out must have q's row count")
+    slots = [int(s) for s in slots]
+    arr = (_I32 * len(slots))(*slots)
+    _check("kv_attention", lib().kv_attention(ctypes.byref(cache._c), layer, arr, len(slots), _ptr(q), tq, ldq,
+                                              float(scale), _ptr(out), ldo, _ptr(status), _stream(stream)))
+    return out
 
 
 def encode_elements(x, stream=None):

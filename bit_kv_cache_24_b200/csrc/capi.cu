@@ -1,12 +1,14 @@
 // capi.cu -- the C ABI declared in include/nvfp4.h: argument validation, layout arithmetic,
 // architecture checks and kernel dispatch.  No allocation, no synchronisation.
 #include <atomic>
+#include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
+#include "attention.h"
 
 namespace nvfp4 {
 
@@ -428,6 +430,56 @@ nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, const int32_
     jv.out = static_cast<uint16_t *>(v_out_bf16);
     cudaError_t e = launch_kv_dequant(&jk, &jv, dev_status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "kv_dequant");
+}
+
+nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, const int32_t *slots, int32_t nslots,
+                          const void *q_bf16, int64_t tq, int64_t ldq, float scale, void *o_bf16, int64_t ldo,
+                          int32_t *dev_status, nvfp4_stream stream) {
+    (void)dev_status;                                     // no data-dependent error exists
+    if (!kv_ok(cache) || !slots || tq < 0 || (tq > 0 && (!q_bf16 || !o_bf16)) || !std::isfinite(scale))
+        return NVFP4_ERR_INVALID_ARG;
+    if (layer < 0 || layer >= cache->layers || nslots <= 0 || nslots > kMaxDequantSlots) return NVFP4_ERR_INVALID_ARG;
+    const int64_t row = (int64_t)cache->heads * cache->head_dim;
+    if (ldq < row || ldo < row) return NVFP4_ERR_INVALID_ARG;
+    if (cache->head_dim != 128 || cache->heads > 65535 || (ldq & 7) || (ldo & 7) || !aligned16(q_bf16) ||
+        !aligned16(o_bf16) || !aligned16(cache->codes_k) || !aligned16(cache->codes_v) ||
+        !aligned16(cache->sf_k) || !aligned16(cache->sf_v))
+        return NVFP4_ERR_UNSUPPORTED;
+    if (ceil_div(tq, 64) > 0x7FFFFFFF) return NVFP4_ERR_UNSUPPORTED;
+    static thread_local AttnJob j;
+    int64_t tok = 0;
+    int32_t n = 0;
+    for (int32_t i = 0; i < nslots; ++i) {
+        const int32_t s = slots[i];
+        if (s < 0 || s >= cache->slots) return NVFP4_ERR_INVALID_ARG;
+        const int64_t slot_index = (int64_t)layer * cache->slots + s;
+        const int32_t len = cache->len[slot_index];
+        if (len < 0 || len > cache->slot_tokens) return NVFP4_ERR_INVALID_ARG;
+        if (len == 0) continue;
+        const int64_t tok0 = slot_index * cache->slot_tokens;
+        j.slot[n] = AttnSlot{cache->codes_k + tok0 * (row / 2), cache->codes_v + tok0 * (row / 2),
+                             cache->sf_k + tok0 * (row / 16), cache->sf_v + tok0 * (row / 16),
+                             cache->g_k + slot_index, cache->g_v + slot_index, tok};
+        tok += len;
+        ++n;
+    }
+    if (tok == 0) return NVFP4_ERR_INVALID_ARG;           // attention over an empty window
+    if (tq == 0) return NVFP4_OK;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    j.nslots = n;
+    j.heads = cache->heads;
+    j.total_tokens = tok;
+    j.row_bytes = row / 2;
+    j.row_sf = row / 16;
+    j.q = static_cast<const uint16_t *>(q_bf16);
+    j.ldq = ldq;
+    j.tq = tq;
+    j.o = static_cast<uint16_t *>(o_bf16);
+    j.ldo = ldo;
+    j.scale_log2 = (float)((double)scale * 1.4426950408889634);   // log2(e)
+    cudaError_t e = launch_kv_attention(j, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "kv_attention");
 }
 
 nvfp4_status nvfp4_encode_elements(const float *in, int64_t n, uint8_t *e2m1_out, uint8_t *e4m3_out,

@@ -226,6 +226,30 @@ NVFP4_API nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, co
                         nvfp4_stream stream);
 
 /*
+ * kv_attention -- softmax attention of BF16 queries over a window of NVFP4 cache slots, with the
+ * restore fused into the kernel's K/V tile loads: the window's BF16 K and V never reach HBM.
+ * LongLive-2.0 restores its NVFP4 KV cache for attention with a parallel dequantization kernel
+ * (d9249.github.io review, section "핵심 아이디어 / 구조 / 동작 방식"); this call computes the
+ * same attention without the restored copy.  For every head h and query row i:
+ *   O[i, h, :] = sum_j softmax_j(scale * q[i, h, :] . k[j, h, :]) v[j, h, :]
+ * over the tokens j of the listed slots (host array `slots`, nslots <= 128, layer `layer`). k and
+ * v are the values kv_dequant restores, BF16(FP32(e2m1 * sf) * g). The slot order changes only
+ * the summation order. No mask.
+ *   q:  [tq, heads, head_dim] BF16 (DEVICE), token row stride ldq elements (e.g. the Q third of
+ *       a fused QKV GEMM output, ldq = 3 * heads * head_dim);
+ *   o:  [tq, heads, head_dim] BF16 (DEVICE), token row stride ldo elements; must not overlap q;
+ *   scale: the softmax scale (commonly 1 / sqrt(head_dim)), finite.
+ * Requires head_dim == 128, ldq and ldo >= heads * head_dim and multiples of 8, q and o 16-byte
+ * aligned, a window of at least one token (else NVFP4_ERR_INVALID_ARG / NVFP4_ERR_UNSUPPORTED).
+ * tq == 0 is a no-op.
+ * Arithmetic: FP32 scores and output accumulation, the probabilities rounded to BF16 for the
+ * P.V product, the output rounded to BF16 (nearest even).
+ */
+NVFP4_API nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, const int32_t *slots,
+                                    int32_t nslots, const void *q_bf16, int64_t tq, int64_t ldq, float scale,
+                                    void *o_bf16, int64_t ldo, int32_t *dev_status, nvfp4_stream stream);
+
+/*
  * nvfp4_quantize_noalloc -- nvfp4_quantize without a workspace: for callers that cannot
  * allocate, such as plugin/enqueue hooks of inference engines and embedded host programs that
  * receive only their input and output buffers and have no allocator or workspace to hand over.
