@@ -57,7 +57,7 @@ PEAK_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustaine
 def parse_args(argv=None):
     p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=3000)
+    p.add_argument("--steps", type=int, default=None, help="timed steps (default 3000; 200 for --op attention)")
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--e2e-steps", type=int, default=40)
@@ -65,7 +65,10 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=15.0)
     p.add_argument("--op", choices=["step", "attention"], default="step",
                    help="step: the QKV chunk step (default); attention: kv_attention over the step's KV window")
-    return p.parse_args(argv)
+    a = p.parse_args(argv)
+    if a.steps is None:
+        a.steps = 200 if a.op == "attention" else 3000
+    return a
 
 
 # ---------------------------------------------------------------------------------- plumbing

@@ -12,9 +12,11 @@
 // k, v = BF16(FP32(e2m1 * sf) * g), the values the restore kernel produces.  No mask.
 //
 // Design (warp-level BF16 MMA, FlashAttention-2 structure):
-//   - CTA = 64 query rows of one head, 4 warps x 16 rows; Q stays in registers as MMA A fragments.
-//   - Per 64-token tile, each thread holds the raw bytes of half a token row of K and of V
-//     (2 x 32 code bytes, 2 x 4 scale bytes) fetched one tile ahead. It dequantizes them into a
+//   - CTA = 128 query rows of one head, 8 warps x 16 rows; Q stays in registers as MMA A
+//     fragments. Each CTA dequantizes its head's whole window once, so more rows per CTA means
+//     less dequantization per FLOP.
+//   - Per 64-token tile, each thread holds the raw bytes of half a token row of K or of V (32
+//     code bytes, 4 scale bytes) fetched one tile ahead. It dequantizes them into a
 //     double-buffered shared-memory tile. Rows are padded to 272 B, so neither the 16-byte
 //     stores nor ldmatrix conflict on banks.
 //   - S = Q K^T runs on mma.sync m16n8k16 with FP32 accumulation. Then an online softmax in
@@ -32,14 +34,14 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kD = 128;                     // head_dim
-constexpr int kBQ = 64;                     // query rows per CTA
+constexpr int kBQ = 128;                    // query rows per CTA
 constexpr int kBK = 64;                     // window tokens per tile
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kPitch = kD * 2 + 16;         // bytes per shared-memory tile row
 constexpr int kTileBytes = kBK * kPitch;
 constexpr int kSmemBytes = 4 * kTileBytes;  // K and V, two buffers each
 
-static_assert(kThreads == 2 * kBK, "a thread loads half a token row of the tile");
+static_assert(kThreads == 4 * kBK, "a thread loads half a token row of K or of V");
 static_assert(kBQ == 16 * (kThreads / 32), "a warp owns 16 query rows");
 
 // y = BF16(FP32(e2m1 * sf) * g) for the 8 codes of one word: the restore's rounding steps (the
@@ -93,33 +95,29 @@ __device__ __forceinline__ void mma_bf16(float c[4], const uint32_t a[4], uint32
                  : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Raw NVFP4 bytes of half a token row (64 elements) of K and of V, and the slot's g.
+// Raw NVFP4 bytes of half a token row (64 elements) of K or of V, and the slot's g.
 struct Raw {
-    uint4 ck[2], cv[2];
-    uint32_t sk, sv;
-    float gk, gv;
+    uint4 c[2];
+    uint32_t sf;
+    float g;
 };
 
-// Fetch window token `tok` (zeros past the end); `si` is the thread's running slot index
-// (tokens only grow, so it only moves forward).
-__device__ __forceinline__ void fetch(const AttnJob &j, int64_t tok, int &si, int head, int hf, Raw &w) {
-    w.ck[0] = w.ck[1] = w.cv[0] = w.cv[1] = make_uint4(0, 0, 0, 0);
-    w.sk = w.sv = 0;
-    w.gk = w.gv = 0.0f;
+// Fetch window token `tok` of K (v == 0) or V (v == 1), zeros past the end; `si` is the
+// thread's running slot index (tokens only grow, so it only moves forward).
+__device__ __forceinline__ void fetch(const AttnJob &j, int64_t tok, int &si, int head, int hf, int v, Raw &w) {
+    w.c[0] = w.c[1] = make_uint4(0, 0, 0, 0);
+    w.sf = 0;
+    w.g = 0.0f;
     if (tok >= j.total_tokens) return;
     while (si + 1 < j.nslots && tok >= j.slot[si + 1].tok_begin) ++si;
     const AttnSlot &s = j.slot[si];
     const int64_t t = tok - s.tok_begin;
+    const uint8_t *codes = v ? s.codes_v : s.codes_k;
     const int64_t cb = t * j.row_bytes + head * (kD / 2) + hf * 32;
-    const int64_t sb = t * j.row_sf + head * (kD / 16) + hf * 4;
-    w.ck[0] = ldg_nc_v4(s.codes_k + cb);
-    w.ck[1] = ldg_nc_v4(s.codes_k + cb + 16);
-    w.cv[0] = ldg_nc_v4(s.codes_v + cb);
-    w.cv[1] = ldg_nc_v4(s.codes_v + cb + 16);
-    w.sk = ldg_nc_u32(s.sf_k + sb);
-    w.sv = ldg_nc_u32(s.sf_v + sb);
-    w.gk = *s.g_k;
-    w.gv = *s.g_v;
+    w.c[0] = ldg_nc_v4(codes + cb);
+    w.c[1] = ldg_nc_v4(codes + cb + 16);
+    w.sf = ldg_nc_u32((v ? s.sf_v : s.sf_k) + t * j.row_sf + head * (kD / 16) + hf * 4);
+    w.g = *(v ? s.g_v : s.g_k);
 }
 
 // Dequantize one half row (8 words of codes, 4 block scales) into shared memory at `dst`.
@@ -132,7 +130,7 @@ __device__ __forceinline__ void put_half(uint32_t dst, const uint4 c[2], uint32_
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_constant__ AttnJob j) {
+__global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_constant__ AttnJob j) {
     extern __shared__ __align__(128) uint8_t smem[];
     griddep_wait();                                       // the cache and q written by earlier kernels
     griddep_launch_dependents();
@@ -157,20 +155,20 @@ __global__ void __launch_bounds__(kThreads, 2) kv_attention_kernel(const __grid_
     for (int n = 0; n < kD / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;   // rows g and g + 8
 
-    const int lr = threadIdx.x & (kBK - 1), hf = threadIdx.x / kBK;   // loader: token row, half
+    // loader: token row, half of it, K or V
+    const int lr = threadIdx.x & (kBK - 1), hf = (threadIdx.x / kBK) & 1, lv = threadIdx.x / (2 * kBK);
     const int mi = lane >> 3, mr = lane & 7;              // ldmatrix: matrix, row within it
     int si = 0;
     Raw w;
-    fetch(j, lr, si, head, hf, w);
+    fetch(j, lr, si, head, hf, lv, w);
     const uint32_t sbase = smem_addr(smem);
     const int64_t ntiles = (j.total_tokens + kBK - 1) / kBK;
     for (int64_t it = 0; it < ntiles; ++it) {
         // Buffer it & 1: every warp finished tile it - 2 (which used it) before passing the
         // barrier of tile it - 1, so it can be overwritten now.
         const uint32_t kb = sbase + (uint32_t)(it & 1) * 2u * kTileBytes, vb = kb + kTileBytes;
-        put_half(kb + lr * kPitch + hf * 128, w.ck, w.sk, w.gk);
-        put_half(vb + lr * kPitch + hf * 128, w.cv, w.sv, w.gv);
-        if (it + 1 < ntiles) fetch(j, (it + 1) * kBK + lr, si, head, hf, w);
+        put_half((lv ? vb : kb) + lr * kPitch + hf * 128, w.c, w.sf, w.g);
+        if (it + 1 < ntiles) fetch(j, (it + 1) * kBK + lr, si, head, hf, lv, w);
         __syncthreads();
 
         // S = Q K^T: 16 rows x 64 tokens per warp
