@@ -46,3 +46,45 @@ def test_argument_errors_are_synchronous():
     assert L.kv_dequant(None, 0, None, 0, None, None, None, None) == nv.NVFP4_ERR_INVALID_ARG
     for s in range(6):
         assert L.nvfp4_status_string(s)
+
+
+def _fake_cache(heads=2, head_dim=128, slots=3, lens=(5, 0, 7)):
+    """A cache descriptor whose arrays are never dereferenced by the argument checks (host
+    buffers stand in for the device arrays; the slot lengths are a real host array)."""
+    buf = (ctypes.c_uint8 * 4096)()
+    base = (ctypes.addressof(buf) + 15) // 16 * 16
+    ln = (ctypes.c_int32 * slots)(*lens)
+    c = nv._KVCache(1, heads, head_dim, slots, 8, base, base, base, base, base, base,
+                    ctypes.cast(ln, ctypes.POINTER(ctypes.c_int32)))
+    return c, buf, ln, base
+
+
+def test_kv_attention_argument_errors():
+    L = nv.lib()
+    c, buf, ln, base = _fake_cache()
+    row = 2 * 128
+    slots = (ctypes.c_int32 * 3)(0, 1, 2)
+
+    def call(cache=c, layer=0, sl=slots, n=3, q=base, tq=4, ldq=row, scale=1.0, o=base, ldo=row):
+        return L.kv_attention(None if cache is None else ctypes.byref(cache), layer, sl, n, q, tq, ldq, scale, o,
+                              ldo, None, None)
+
+    inv, uns = nv.NVFP4_ERR_INVALID_ARG, nv.NVFP4_ERR_UNSUPPORTED
+    assert call(cache=None) == inv
+    assert call(layer=-1) == inv and call(layer=1) == inv
+    assert call(n=0) == inv and call(n=129) == inv
+    assert call(sl=(ctypes.c_int32 * 3)(0, 3, 2)) == inv          # slot id out of range
+    assert call(tq=-1) == inv
+    assert call(scale=float("inf")) == inv and call(scale=float("nan")) == inv
+    assert call(ldq=row - 8) == inv and call(ldo=row - 8) == inv
+    assert call(q=None) == inv and call(o=None) == inv
+    assert call(ldq=row + 4) == uns                                # row stride not a multiple of 8
+    assert call(q=base + 2) == uns and call(o=base + 8) == uns     # not 16-byte aligned
+    assert call(sl=(ctypes.c_int32 * 1)(1), n=1) == inv            # empty window
+    ln[0] = 9                                                      # longer than a slot holds
+    assert call() == inv
+    ln[0] = 5
+    # no queries: nothing to launch, even with no q/o buffers
+    assert call(tq=0, q=None, o=None) == nv.NVFP4_OK
+    c64, buf64, ln64, base64 = _fake_cache(head_dim=64)
+    assert L.kv_attention(ctypes.byref(c64), 0, slots, 3, base64, 4, 128, 1.0, base64, 128, None, None) == uns
