@@ -241,7 +241,8 @@ NVFP4_API nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, co
  *   scale: the softmax scale (commonly 1 / sqrt(head_dim)), finite.
  * Requires head_dim == 128, ldq and ldo >= heads * head_dim and multiples of 8, q and o 16-byte
  * aligned, a window of at least one token (else NVFP4_ERR_INVALID_ARG / NVFP4_ERR_UNSUPPORTED).
- * tq == 0 is a no-op.
+ * tq == 0 is a no-op. dev_status may be NULL: the kernel has no data-dependent error (it never
+ * waits), and scores must stay finite in FP32 (|scale * q.k| < 2^127) for a finite result.
  * Arithmetic: FP32 scores and output accumulation, the probabilities rounded to BF16 for the
  * P.V product, the output rounded to BF16 (nearest even).
  */
