@@ -63,11 +63,12 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=40)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
-    p.add_argument("--op", choices=["step", "attention"], default="step",
-                   help="step: the QKV chunk step (default); attention: kv_attention over the step's KV window")
+    p.add_argument("--op", choices=["step", "attention", "appends"], default="step",
+                   help="step: the QKV chunk step (default); attention: kv_attention over the step's KV "
+                        "window; appends: one chunk's KV append into all 30 layers, as a CUDA graph")
     a = p.parse_args(argv)
     if a.steps is None:
-        a.steps = 200 if a.op == "attention" else 3000
+        a.steps = {"attention": 200, "appends": 300}.get(a.op, 3000)
     return a
 
 
@@ -646,6 +647,92 @@ def attention_cpu_baseline(seconds, rows=4):
             "sample": f"{n} calls of {rows} query rows x 1 head over the 56160-token window in {dt:.1f} s"}
 
 
+# ------------------------------------------------------------------------------ appends op
+
+LAYERS = 30
+APPEND_BYTES = 2 * M_TOK * HEADS * HEAD_DIM * (2 + 0.5 + 1 / 16)   # K and V: BF16 in, codes + scales out
+
+
+def run_appends(args, rank, local_rank, world):
+    """One chunk's KV append into every layer of a 30-layer cache (kv_quant_append per layer,
+    three kernels each), launched back to back and, separately, replayed as one CUDA graph.
+    A step is all 30 appends. The K/V inputs rotate over 6 distinct layers' tensors (345 MB,
+    more than the 126 MB L2)."""
+    import bit_kv_cache_24_b200 as nv
+    from bit_kv_cache_24_b200 import synth
+    dist = init_dist(world, "nccl")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cache = nv.KVCache(LAYERS, HEADS, HEAD_DIM, 1, M_TOK, dev)
+    kv = [tuple(t.to(dev) for t in synth.kv_chunk(layer, 0)) for layer in range(6)]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+
+    def appends():
+        for layer in range(LAYERS):
+            k, v = kv[layer % len(kv)]
+            nv.kv_quant_append(cache, layer, 0, k, v, status=status)
+
+    for _ in range(max(args.warmup, 3)):                  # also sets every launch attribute once
+        appends()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        appends()
+    torch.cuda.synchronize()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    if dist:
+        dist.barrier()
+    clocks = ClockSampler(local_rank)
+    ev[0].record(stream)
+    for _ in range(K):
+        graph.replay()
+    ev[1].record(stream)
+    for _ in range(K):
+        appends()
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    graph_s = reduce_max(ev[0].elapsed_time(ev[1]) / 1e3, dist, dev)
+    eager_s = reduce_max(ev[1].elapsed_time(ev[2]) / 1e3, dist, dev)
+    peaks, src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", PEAK_FALLBACK["hbm_gbs"]))
+    gbs = APPEND_BYTES * LAYERS * K / graph_s / 1e9
+    line = {
+        "metric": "KV append GB/s (30 layers per step, CUDA graph; % of HBM peak)",
+        "value": round(aggregate(APPEND_BYTES * LAYERS * K / 1e9, world, graph_s), 1), "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": round(graph_s * 1e3 / K, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 -> nvfp4 (e2m1 x e4m3/16)", "data": "synthetic (seeded; K/V of the KV workload)",
+        "config": {"workload": "kv_quant_append of one 4680-token chunk (24 heads x 128, K and V) into each "
+                               "of 30 layers", "global_batch": M_TOK * world, "seq_len": M_TOK,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs rotate over 6 layers' K/V (345 MB) > 126 MB L2"},
+        "gpu_launches": 3 * LAYERS * 2 * K,
+        "eager": {"ms_per_step": round(eager_s * 1e3 / K, 4),
+                  "value": round(APPEND_BYTES * LAYERS * K / eager_s / 1e9, 1), "unit": "GB/s"},
+        "roofline": {"kernel": "kv_quant_append (amax, scale record, row pass)", "bound": "hbm",
+                     "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s", "frac": round(gbs / hbm, 4),
+                     "traffic": None, "peak_source": f"{src} (HBM copy)"},
+        "clocks": clk,
+        "device_status": int(status.item()),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, local_rank, world = dist_env()
@@ -654,6 +741,9 @@ def main(argv=None):
         return
     if args.op == "attention":
         run_attention(args, rank, local_rank, world)
+        return
+    if args.op == "appends":
+        run_appends(args, rank, local_rank, world)
         return
     run_ours(args, rank, local_rank, world)
 
