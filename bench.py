@@ -63,12 +63,13 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=40)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
-    p.add_argument("--op", choices=["step", "attention", "appends"], default="step",
+    p.add_argument("--op", choices=["step", "attention", "appends", "kernels"], default="step",
                    help="step: the QKV chunk step (default); attention: kv_attention over the step's KV "
-                        "window; appends: one chunk's KV append into all 30 layers, as a CUDA graph")
+                        "window; appends: one chunk's KV append into all 30 layers, as a CUDA graph; "
+                        "kernels: every kernel standalone on every workload shape (cold L2)")
     a = p.parse_args(argv)
     if a.steps is None:
-        a.steps = {"attention": 200, "appends": 300}.get(a.op, 3000)
+        a.steps = {"attention": 200, "appends": 300, "kernels": 20}.get(a.op, 3000)
     return a
 
 
@@ -733,6 +734,130 @@ def run_appends(args, rank, local_rank, world):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------------------ kernels op
+
+def run_kernels(args, rank, local_rank, world):
+    """Every kernel standalone on the workload shapes: L2 flushed (a 256 MB read) before each
+    launch, the host enqueue hidden behind a device sleep, median of `--steps` launches (20 by
+    default). Beside each NVFP4 GEMM, cuBLASLt's NVFP4 GEMM (torch scaled_mm) on the same quantized
+    operands, as library context; it is not part of the path."""
+    import bit_kv_cache_24_b200 as nv
+    from bit_kv_cache_24_b200 import synth
+    if world > 1:
+        raise SystemExit("--op kernels runs on one GPU")
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    reps = args.steps
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+    def timeit(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.max()
+            torch.cuda._sleep(2_000_000)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b) / 1e3)
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    peaks, src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", PEAK_FALLBACK["hbm_gbs"]))
+    fp4 = float(peaks.get("bf16_tflops", PEAK_FALLBACK["bf16_tflops"])) * FP4_OVER_BF16
+    out = {}
+
+    def lib_gemm(A, B, y_ref):
+        """cuBLASLt NVFP4 GEMM through torch on our codes and tensor-core scales; returns the
+        context entry (time, or why it is unavailable)."""
+        import torch.nn.functional as F
+        M, N, K = A.rows, B.rows, A.cols
+        try:
+            a = A.codes.view(torch.float4_e2m1fn_x2)
+            b = B.codes.view(torch.float4_e2m1fn_x2).t()
+            sa = A.sf.view(torch.float8_e4m3fn).view(128 * ((M + 127) // 128), -1)
+            sb = B.sf.view(torch.float8_e4m3fn).view(128 * ((N + 127) // 128), -1)
+            ST, SW = F.ScalingType, F.SwizzleType
+            call = lambda: F.scaled_mm(a, b, [sa, A.g], [ST.BlockWise1x16, ST.TensorWise], [sb, B.g],
+                                       [ST.BlockWise1x16, ST.TensorWise], swizzle_a=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE],
+                                       swizzle_b=[SW.SWIZZLE_32_4_4, SW.NO_SWIZZLE], output_dtype=torch.bfloat16)
+            y = call()
+            torch.cuda.synchronize()
+            rel = float((y.float() - y_ref.float()).norm() / y_ref.float().norm().clamp_min(1e-30))
+            if not rel < 1e-2:
+                return {"unavailable": f"result differs from ours (rel. Frobenius {rel:.3g})"}
+            t = timeit(call)
+            return {"us": round(t * 1e6, 1), "tflops": round(2 * M * N * K / t / 1e12, 1), "rel_frobenius_vs_ours": rel}
+        except Exception as e:                            # library context only
+            return {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:160]}"}
+
+    def gemm(name, A, B, bias=None, resid=None):
+        y = torch.empty(A.rows, B.rows, dtype=torch.bfloat16, device=dev)
+        run = lambda: nv.nvfp4_gemm(A, B, bias=bias, resid=resid, out=y)
+        t = timeit(run)
+        tf = 2 * A.rows * B.rows * A.cols / t / 1e12
+        y0 = nv.nvfp4_gemm(A, B)                          # no epilogue term: what the library call computes
+        out[f"gemm_{name}"] = {"shape": [A.rows, B.rows, A.cols], "us": round(t * 1e6, 1), "tflops": round(tf, 1),
+                               "frac_fp4_ref": round(tf / fp4, 4), "cublaslt_nvfp4": lib_gemm(A, B, y0)}
+
+    def quant(name, x):
+        M, K = x.shape
+        byt = M * K * (2 + 0.5 + 1 / 16)
+        A = nv.nvfp4_quantize(x)
+        amax = nv.nvfp4_amax(x)
+        Ac = nv.nvfp4_quantize(x, nv.COLWISE)
+        e = {"shape": [M, K]}
+        for key, fn in (("two_pass", lambda: nv.nvfp4_quantize(x, out=A)),
+                        ("row_amax_given", lambda: nv.nvfp4_quantize(x, amax_in=amax, out=A)),
+                        ("col_amax_given", lambda: nv.nvfp4_quantize(x, nv.COLWISE, amax_in=amax, out=Ac))):
+            t = timeit(fn)
+            e[key] = {"us": round(t * 1e6, 1), "gbs": round(byt / t / 1e9, 1), "frac_hbm": round(byt / t / 1e9 / hbm, 4)}
+        out[f"quantize_{name}"] = e
+
+    d = {k: v.to(dev) for k, v in synth.qkv().items()}
+    quant("qkv_A", d["A"])
+    quant("qkv_W", d["W"])
+    gemm("qkv", nv.nvfp4_quantize(d["A"]), nv.nvfp4_quantize(d["W"]), bias=d["bias"])
+    d = {k: v.to(dev) for k, v in synth.ffn().items()}
+    quant("ffn_down_A", d["A_down"])
+    gemm("ffn_up", nv.nvfp4_quantize(d["A_up"]), nv.nvfp4_quantize(d["W_up"]))
+    gemm("ffn_down", nv.nvfp4_quantize(d["A_down"]), nv.nvfp4_quantize(d["W_down"]), resid=d["R"])
+    d = {k: v.to(dev) for k, v in synth.train().items()}
+    quant("train_X", d["X"])
+    X, dY, W = nv.nvfp4_quantize(d["X"]), nv.nvfp4_quantize(d["dY"]), nv.nvfp4_quantize(d["W"])
+    gemm("fprop", X, W)
+    gemm("dgrad", dY, nv.nvfp4_quantize(d["W"], nv.COLWISE))
+    gemm("wgrad", nv.nvfp4_quantize(d["dY"], nv.COLWISE), nv.nvfp4_quantize(d["X"], nv.COLWISE))
+    del d, X, dY, W
+    sq = synth.ragged(8192, 8192, 8192).to(dev)
+    gemm("8192cubed", nv.nvfp4_quantize(sq), nv.nvfp4_quantize(sq))
+    del sq
+
+    cache = nv.KVCache(1, HEADS, HEAD_DIM, SLOTS, M_TOK, dev)
+    chunks = [tuple(t.to(dev) for t in synth.kv_chunk(0, s)) for s in range(SLOTS)]
+    for s, (k, v) in enumerate(chunks):
+        nv.kv_quant_append(cache, 0, s, k, v)
+    kout = torch.empty(SLOTS * M_TOK, HEADS, HEAD_DIM, dtype=torch.bfloat16, device=dev)
+    vout = torch.empty_like(kout)
+    t = timeit(lambda: nv.kv_dequant(cache, 0, list(range(SLOTS)), k_out=kout, v_out=vout))
+    byt = 2 * SLOTS * M_TOK * HEADS * HEAD_DIM * (0.5 + 1 / 16 + 2)
+    out["kv_dequant_window"] = {"us": round(t * 1e6, 1), "gbs": round(byt / t / 1e9, 1),
+                                "frac_hbm": round(byt / t / 1e9 / hbm, 4)}
+    k, v = chunks[0]
+    t = timeit(lambda: nv.kv_quant_append(cache, 0, 0, k, v))
+    byt = APPEND_BYTES
+    out["kv_append_chunk"] = {"us": round(t * 1e6, 1), "gbs": round(byt / t / 1e9, 1),
+                              "frac_hbm": round(byt / t / 1e9 / hbm, 4)}
+    line = {"metric": "standalone kernel timings (L2 flushed, median)", "unit": "us", "reps": reps,
+            "peaks": {"hbm_gbs": hbm, "fp4_ref_tflops_burst": fp4, "source": src},
+            "data": "synthetic (seeded workload generators)", "kernels": out}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     rank, local_rank, world = dist_env()
@@ -744,6 +869,9 @@ def main(argv=None):
         return
     if args.op == "appends":
         run_appends(args, rank, local_rank, world)
+        return
+    if args.op == "kernels":
+        run_kernels(args, rank, local_rank, world)
         return
     run_ours(args, rank, local_rank, world)
 
