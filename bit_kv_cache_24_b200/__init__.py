@@ -87,6 +87,8 @@ def lib():
             "kv_quant_append_amax": (_I32, [ctypes.POINTER(_KVCache), _I32, _I32, _P, _P, _I64, _I64, _P, _P, _SZ, _P,
                                             _P]),
             "kv_dequant": (_I32, [ctypes.POINTER(_KVCache), _I32, ctypes.POINTER(_I32), _I32, _P, _P, _P, _P]),
+            "nvfp4_sf_to_linear": (_I32, [_P, _I64, _I64, _P]),
+            "nvfp4_sf_to_mma": (_I32, [_P, _I64, _I64, _P]),
             "kv_attention": (_I32, [ctypes.POINTER(_KVCache), _I32, ctypes.POINTER(_I32), _I32, _P, _I64, _I64,
                                     ctypes.c_float, _P, _I64, _P, _P]),
             "nvfp4_encode_elements": (_I32, [_P, _I64, _P, _P, _P]),
@@ -331,6 +333,16 @@ def kv_attention(cache: KVCache, layer, slots, q, scale, out=None, status=None, 
     arr = (_I32 * len(slots))(*slots)
     _check("kv_attention", lib().kv_attention(ctypes.byref(cache._c), layer, arr, len(slots), _ptr(q), tq, ldq,
                                               float(scale), _ptr(out), ldo, _ptr(status), _stream(stream)))
+    return out
+
+
+def sf_to_linear(q: QTensor) -> torch.Tensor:
+    """The scales of q as a host [rows, ceil(cols/16)] uint8 table (linear layout)."""
+    sf = q.sf.cpu().contiguous()
+    if q.sf_layout == SF_LINEAR:
+        return sf.view(q.rows, -1)
+    out = torch.empty(q.rows, (q.cols + 15) // 16, dtype=torch.uint8)
+    _check("nvfp4_sf_to_linear", lib().nvfp4_sf_to_linear(_ptr(sf), q.rows, q.cols, _ptr(out)))
     return out
 
 

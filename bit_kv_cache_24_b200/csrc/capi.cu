@@ -153,6 +153,23 @@ int64_t nvfp4_codes_pitch(int64_t cols) { return cols < 0 ? -1 : codes_pitch(col
 
 int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols, int32_t layout) { return sf_bytes(rows, cols, layout); }
 
+nvfp4_status nvfp4_sf_to_linear(const uint8_t *sf_mma, int64_t rows, int64_t cols, uint8_t *sf_linear) {
+    if (!sf_mma || !sf_linear || rows <= 0 || cols <= 0) return NVFP4_ERR_INVALID_ARG;
+    const int64_t nb = ceil_div(cols, 16), apr = ceil_div(nb, 4);
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t b = 0; b < nb; ++b) sf_linear[i * nb + b] = sf_mma[sf_mma_offset(i, b, apr)];
+    return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_sf_to_mma(const uint8_t *sf_linear, int64_t rows, int64_t cols, uint8_t *sf_mma) {
+    if (!sf_mma || !sf_linear || rows <= 0 || cols <= 0) return NVFP4_ERR_INVALID_ARG;
+    const int64_t nb = ceil_div(cols, 16), apr = ceil_div(nb, 4);
+    memset(sf_mma, 0, (size_t)sf_bytes(rows, cols, NVFP4_SF_MMA));
+    for (int64_t i = 0; i < rows; ++i)
+        for (int64_t b = 0; b < nb; ++b) sf_mma[sf_mma_offset(i, b, apr)] = sf_linear[i * nb + b];
+    return NVFP4_OK;
+}
+
 size_t nvfp4_quantize_workspace(int64_t rows, int64_t cols) {
     (void)rows;
     (void)cols;

@@ -103,6 +103,15 @@ NVFP4_API int64_t nvfp4_codes_pitch(int64_t cols);
 /* Bytes of the scale array of a rows x cols matrix in `layout`; -1 on bad arguments. */
 NVFP4_API int64_t nvfp4_sf_bytes(int64_t rows, int64_t cols, int32_t layout);
 
+/* Scale layout conversion on HOST memory (no device work), e.g. to read the tensor-core scale
+ * layout of a GEMM operand as a plain table.
+ * nvfp4_sf_to_linear: sf_mma (nvfp4_sf_bytes(rows, cols, NVFP4_SF_MMA) bytes) -> sf_linear
+ * ([rows][ceil(cols/16)] bytes); the layout's padding is dropped.
+ * nvfp4_sf_to_mma: the inverse, with the padding rows and scale columns written as zero.
+ * NVFP4_ERR_INVALID_ARG on a NULL pointer or rows, cols <= 0. */
+NVFP4_API nvfp4_status nvfp4_sf_to_linear(const uint8_t *sf_mma, int64_t rows, int64_t cols, uint8_t *sf_linear);
+NVFP4_API nvfp4_status nvfp4_sf_to_mma(const uint8_t *sf_linear, int64_t rows, int64_t cols, uint8_t *sf_mma);
+
 /* Bytes of device workspace nvfp4_quantize / nvfp4_amax need (per-CTA partial maxima and the
  * per-tensor scale record; 5 KB). */
 NVFP4_API size_t nvfp4_quantize_workspace(int64_t rows, int64_t cols);

@@ -3,9 +3,12 @@ declares, its size arithmetic agrees with the oracle's independent layout code, 
 errors are rejected before any device work."""
 import ctypes
 
+import numpy as np
 import pytest
+import torch
 
 import bit_kv_cache_24_b200 as nv
+from bit_kv_cache_24_b200 import synth
 
 
 def test_library_exports_every_header_function():
@@ -88,3 +91,32 @@ def test_kv_attention_argument_errors():
     assert call(tq=0, q=None, o=None) == nv.NVFP4_OK
     c64, buf64, ln64, base64 = _fake_cache(head_dim=64)
     assert L.kv_attention(ctypes.byref(c64), 0, slots, 3, base64, 4, 128, 1.0, base64, 128, None, None) == uns
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 16), (3, 17), (128, 256), (130, 96), (300, 512), (4680, 3072)])
+def test_scale_layout_conversion_matches_oracle(orc, rows, cols):
+    L = nv.lib()
+    nb = (cols + 15) // 16
+    lin = np.random.default_rng(rows * 7 + cols).integers(0, 256, size=rows * nb, dtype=np.uint8)
+    mma = np.full(L.nvfp4_sf_bytes(rows, cols, nv.SF_MMA), 0xAB, dtype=np.uint8)   # padding must be zeroed
+    assert L.nvfp4_sf_to_mma(lin.ctypes.data, rows, cols, mma.ctypes.data) == nv.NVFP4_OK
+    assert np.array_equal(mma, orc.sf_linear_to_mma(lin, rows, cols))        # the oracle's own layout code
+    back = np.zeros(rows * nb, dtype=np.uint8)
+    assert L.nvfp4_sf_to_linear(mma.ctypes.data, rows, cols, back.ctypes.data) == nv.NVFP4_OK
+    assert np.array_equal(back, lin)
+
+
+def test_scale_layout_conversion_argument_errors():
+    L = nv.lib()
+    buf = (ctypes.c_uint8 * 512)()
+    assert L.nvfp4_sf_to_linear(None, 4, 32, buf) == nv.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_sf_to_mma(buf, 0, 32, buf) == nv.NVFP4_ERR_INVALID_ARG
+    assert L.nvfp4_sf_to_mma(buf, 4, -1, buf) == nv.NVFP4_ERR_INVALID_ARG
+
+
+def test_sf_to_linear_of_a_host_qtensor(orc):
+    x = synth.ragged(3, 200, 96, "wide")
+    _, ref = orc.quantize(x)
+    q = nv.QTensor(200, 96, nv.SF_MMA, "cpu")
+    q.sf.copy_(torch.from_numpy(orc.sf_linear_to_mma(ref.sf.reshape(-1), 200, 96)))
+    assert np.array_equal(nv.sf_to_linear(q).numpy(), ref.sf.reshape(200, -1))
