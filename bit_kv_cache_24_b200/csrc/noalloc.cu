@@ -10,9 +10,9 @@
 // Contract:
 //   - The scratch is 5 KB of static device memory (1024 32-bit partial slots and one scale
 //     record), held by every GPU that loads the library until the process exits.
-//   - A call needs one slot per CTA of the amax pass; on GPUs with up to 256 SMs every shape
-//     fits.  A launch that would need more slots is rejected with NVFP4_ERR_UNSUPPORTED and a
-//     message in nvfp4_last_error(); a failed CUDA call returns NVFP4_ERR_CUDA, likewise.
+//   - A call needs one slot per CTA of the amax pass, whose grid is capped at 1024 CTAs, so
+//     every shape fits.  A failed CUDA call returns NVFP4_ERR_CUDA with a message in
+//     nvfp4_last_error().
 //   - All calls share the one array and it keeps the last call's contents.  Nothing in it needs
 //     to start at zero: each call's amax pass writes every slot its record kernel reads, and the
 //     record kernel writes the whole record its quantize pass reads.  Calls
@@ -20,6 +20,8 @@
 //     threads) race on the array and give wrong results; order them on one stream.
 //   - The first call on each device looks up the array's device address (cudaGetSymbolAddress,
 //     with that device current) and caches it; make that first call before any stream capture.
+//     The cached address stays valid as long as the device's primary context lives: a caller
+//     that resets the device (cudaDeviceReset) must not call this entry point afterwards.
 #include <cstdio>
 #include <mutex>
 
@@ -87,7 +89,7 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, in
     if (major != 10 || minor != 0) return NVFP4_ERR_UNSUPPORTED;
 
     const int npartial = amax_blocks(M);
-    if (npartial > kNoAllocPartials) {
+    if (npartial > kNoAllocPartials) {   // static guard: amax_blocks() never exceeds kMaxPartials
         char msg[160];
         std::snprintf(msg, sizeof(msg),
                       "nvfp4_quantize_noalloc: the amax pass needs %d scratch slots, the static scratch holds %d",

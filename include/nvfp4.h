@@ -86,7 +86,13 @@ typedef struct {
  *   sf_k/v:    [layers][slots][slot_tokens][heads*head_dim/16] bytes     (device)
  *   g_k/v:     [layers][slots] floats                                    (device)
  *   len:       [layers][slots] int32 tokens held per slot                (HOST; written by
- *              kv_quant_append, read by kv_dequant) */
+ *              kv_quant_append, read by kv_dequant and kv_attention)
+ * Ordering: `len` is host bookkeeping, read and written when a call is ENQUEUED, not when its
+ * kernels run.  kv_quant_append sets len[slot] before it returns, i.e. before the slot's bytes
+ * exist on the device; a later kv_dequant / kv_attention sizes its launch from it at once.  So
+ * a call that reads a slot must be enqueued after the append that wrote it, on the same stream
+ * or on a stream that waits for an event recorded after the append.  An append that returns an
+ * error leaves len unchanged. */
 typedef struct {
     int32_t layers, heads, head_dim, slots, slot_tokens;
     uint8_t *codes_k, *codes_v;
@@ -133,6 +139,11 @@ NVFP4_API nvfp4_status nvfp4_amax(const void *x_bf16, int64_t M, int64_t K, int6
 
 /*
  * nvfp4_quantize -- BF16 [M, K] (row stride ld elements, K % 8 == 0) to NVFP4.
+ * Defining passage: the LongLive-2.0 arXiv abstract (fugumt.com page) -- the linear layers run
+ * "W4A4 NVFP4" in inference and NVFP4 GEMMs in training, so every activation (and, once, every
+ * weight) is quantized to NVFP4; the d9249.github.io review, section "핵심 아이디어 / 구조 / 동작
+ * 방식", for NVFP4 training and W4A4 inference.  The numeric format is the published NVFP4 one
+ * (top of this file); the pages do not define it.
  *   dir = NVFP4_ROWWISE: 16-blocks along K (the contiguous dim); out->rows = M, out->cols = K.
  *         Requires K % 16 == 0.
  *   dir = NVFP4_COLWISE: 16-blocks along M (the token dim), i.e. the row-wise quantization of
@@ -152,6 +163,10 @@ NVFP4_API nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, 
                             size_t ws_bytes, int32_t *dev_status, nvfp4_stream stream);
 
 /*
+ * Defining passage: the LongLive-2.0 arXiv abstract (fugumt.com page) -- W4A4 NVFP4 linear layers
+ * in inference and NVFP4-accelerated GEMMs in training, whose share of the DiT's work grows with
+ * video length (d9249.github.io review, section "핵심 아이디어 / 구조 / 동작 방식", and its
+ * Table 1 training times).
  * nvfp4_gemm -- Y[M, N] = alpha * A . B^T (+ bias[n] | + resid[m, n]), alpha = gA * gB, with
  * A = [M, K] and B = [N, K] NVFP4 (both K-major, scales in NVFP4_SF_MMA layout) and FP32
  * accumulation in tensor memory (tcgen05 block-scaled MMA, kind::mxf4nvf4).  Epilogue in FP32:
@@ -202,6 +217,9 @@ NVFP4_API int64_t nvfp4_kv_cache_bytes(int32_t layers, int32_t heads, int32_t he
                              int32_t slot_tokens, int32_t which);
 
 /*
+ * Defining passage: the LongLive-2.0 arXiv abstract (fugumt.com page) keeps the KV cache in NVFP4
+ * to cut memory (Table 3 of the paper, as the d9249.github.io review reports it: 29.7 -> 19.4 GB);
+ * the yourai.pro report lists in-place updates of the quantized cache data.
  * kv_quant_append -- quantize one chunk's K and V ([ntok, heads*head_dim] BF16, row stride ld
  * elements; e.g. slices of a fused QKV GEMM output) into slot `slot` of layer `layer`, in place:
  * nothing else in the cache is touched and older slots are never re-quantized.  Each of K and V
@@ -226,6 +244,9 @@ NVFP4_API nvfp4_status kv_quant_append_amax(nvfp4_kv_cache *cache, int32_t layer
                                   nvfp4_stream stream);
 
 /*
+ * Defining passage: the d9249.github.io review, section "핵심 아이디어 / 구조 / 동작 방식" -- the
+ * NVFP4 KV cache is restored by a parallel dequantization kernel to lower the restore cost; the
+ * yourai.pro report lists faster FP4 dequantization among the inference-path optimizations.
  * kv_dequant -- parallel restore of a window of slots of one layer to BF16: the listed slots
  * (host array `slots`, nslots <= 128, in the given order) are dequantized and concatenated
  * token-wise into k_out / v_out ([sum of len, heads, head_dim] BF16, contiguous).
@@ -264,14 +285,16 @@ NVFP4_API nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, 
  * allocate, such as plugin/enqueue hooks of inference engines and embedded host programs that
  * receive only their input and output buffers and have no allocator or workspace to hand over.
  * No counterpart in the paper: it is a deployment variant of the quantizer above.
- * Same arguments, layouts and results as nvfp4_quantize with amax_in = NULL, bit for bit; the
- * amax partial maxima (1024 slots) and the scale record go to a 5 KB static device array held
- * by every GPU that loads the library.  Nothing is allocated.  A launch needing more than 1024
- * slots (only possible on GPUs with more than 256 SMs) returns NVFP4_ERR_UNSUPPORTED with a
- * message in
- * nvfp4_last_error().  All calls share the array: calls whose kernels overlap on the GPU race
- * and must be ordered on one stream.  The first call on each device looks up the array's device
- * address; make that first call before any stream capture.
+ * Accepts dir = NVFP4_ROWWISE or NVFP4_COLWISE only (NVFP4_ROWCOL returns
+ * NVFP4_ERR_INVALID_ARG) and a single output tensor `out`; otherwise the same arguments, layouts
+ * and results as nvfp4_quantize with amax_in = NULL, bit for bit.  The amax partial maxima and
+ * the scale record go to a 5 KB static device array held by every GPU that loads the library.
+ * Nothing is allocated.  The amax pass never launches more than 1024 CTAs, so every shape fits
+ * the array's 1024 partial slots.  All calls share the array: calls whose kernels overlap on the
+ * GPU race and must be ordered on one stream.  The first call on each device looks up the
+ * array's device address and caches it for the life of the process; make that first call before
+ * any stream capture.  The cache assumes the device's primary context is never reset
+ * (cudaDeviceReset) while the library is loaded.
  */
 NVFP4_API nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, int64_t ld, int32_t dir,
                                               const nvfp4_tensor *out, int32_t *dev_status,

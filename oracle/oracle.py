@@ -250,6 +250,36 @@ def gemm_rows(A: Quantized, B: Quantized, rows=None, bias=None, resid=None, thre
     return y
 
 
+def gemm_full(A: Quantized, B: Quantized, bias=None, resid=None):
+    """fp64 reference of every output, Y[M, N] = Adeq . Bdeq^T (+bias | +resid), for sizes where
+    the per-row loop of gemm_rows would take hours on the host (K = 37440, 115 M outputs).
+
+    Same definition as gemm_rows: the dequantized operands are exact in fp64 (dequant_f64), and
+    the contraction is one library step, numpy's fp64 matmul.  Only the fp64 summation order
+    differs from the plain sequential sum (relative differences ~1e-16 * sqrt(K), far below the
+    1e-5 GEMM tolerance); tests/test_oracle_gemm.py checks the two against each other."""
+    assert A.cols == B.cols
+    y = dequant_f64(A) @ dequant_f64(B).T
+    if bias is not None:
+        y += bf16_bits_to_f32(as_u16(bias)).astype(np.float64)[None, :]
+    if resid is not None:
+        y += bf16_bits_to_f32(as_u16(resid)).astype(np.float64)
+    return y
+
+
+def bf16_from_f64(y) -> np.ndarray:
+    """BF16 bits (uint16) of fp64 values rounded once, to nearest with ties to even (8 significant
+    bits), without the detour through FP32 that would round twice.  Finite values in the BF16
+    normal range; values beyond the BF16 range map to +-inf.  Used to compare a BF16 GEMM output
+    with the rounding of the exact result."""
+    y = np.asarray(y, dtype=np.float64)
+    m, e = np.frexp(y)                                    # y = m * 2^e, 0.5 <= |m| < 1
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)          # rint: ties to even
+    with np.errstate(over="ignore"):
+        f = r.astype(np.float32)                          # exact: 8 significant bits
+    return (f.view(np.uint32) >> 16).astype(np.uint16)
+
+
 # ---- KV cache model --------------------------------------------------------------------------
 
 class KVCacheModel:

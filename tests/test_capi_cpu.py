@@ -120,3 +120,26 @@ def test_sf_to_linear_of_a_host_qtensor(orc):
     q = nv.QTensor(200, 96, nv.SF_MMA, "cpu")
     q.sf.copy_(torch.from_numpy(orc.sf_linear_to_mma(ref.sf.reshape(-1), 200, 96)))
     assert np.array_equal(nv.sf_to_linear(q).numpy(), ref.sf.reshape(200, -1))
+
+
+def test_kv_append_that_fails_leaves_slot_length_unchanged():
+    """The cache's per-slot token counts are host bookkeeping written when an append is enqueued
+    (the ordering rule of nvfp4_kv_cache.len): an append that returns an error, whether from its
+    argument checks or (on this GPU-less host) from the device check, must not touch them."""
+    L = nv.lib()
+    c, buf, ln, base = _fake_cache(heads=2, head_dim=128, slots=3, lens=(5, 0, 7))
+    ws = (ctypes.c_uint8 * (L.nvfp4_kv_append_workspace(8, 2, 128) + 16))()
+    wsp = (ctypes.addressof(ws) + 15) // 16 * 16
+    row = 2 * 128
+
+    def append(slot, ntok, ld=row, k=base):
+        return L.kv_quant_append(ctypes.byref(c), 0, slot, k, base, ntok, ld, wsp,
+                                 L.nvfp4_kv_append_workspace(8, 2, 128), None, None)
+
+    assert append(1, 9) == nv.NVFP4_ERR_INVALID_ARG               # more tokens than a slot holds
+    assert append(3, 4) == nv.NVFP4_ERR_INVALID_ARG               # slot out of range
+    assert append(1, 4, ld=row + 4) == nv.NVFP4_ERR_UNSUPPORTED   # row stride not a multiple of 8
+    assert append(1, 4, k=base + 2) == nv.NVFP4_ERR_UNSUPPORTED   # K not 16-byte aligned
+    if not torch.cuda.is_available():
+        assert append(1, 4) in (nv.NVFP4_ERR_CUDA, nv.NVFP4_ERR_UNSUPPORTED)   # no device here
+    assert list(ln) == [5, 0, 7]

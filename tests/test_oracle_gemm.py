@@ -79,3 +79,53 @@ def test_gemm_bias_residual_and_row_subset(orc):
     rows = np.array([11, 0, 5])
     ys = orc.gemm_rows(qa, qb, rows=rows, resid=resid)
     assert np.array_equal(ys, yr[rows])
+
+
+@pytest.mark.parametrize("M,N,K,extra", [(37, 40, 96, None), (130, 24, 544, "bias"), (64, 16, 1008, "resid")])
+def test_gemm_full_equals_the_row_loop(orc, M, N, K, extra):
+    """gemm_full (one fp64 matmul of the dequantized operands, for full-size outputs) against the
+    plain per-element sequential sum of gemm_rows: only the fp64 summation order differs."""
+    a = synth.ragged(M + 2 * K, M, K, "outliers")
+    w = synth.ragged(N + 5 * K, N, K, "lognormal")
+    _, qa = orc.quantize(a)
+    _, qb = orc.quantize(w)
+    kw = {}
+    if extra == "bias":
+        kw["bias"] = synth.ragged(8, 1, N, "normal")[0]
+    elif extra == "resid":
+        kw["resid"] = synth.ragged(9, M, N, "normal")
+    full = orc.gemm_full(qa, qb, **kw)
+    rows = orc.gemm_rows(qa, qb, **kw)
+    scale = np.abs(_deq(qa)).max() * np.abs(_deq(qb)).max() * K
+    assert full.shape == (M, N)
+    assert np.max(np.abs(full - rows)) <= 1e-12 * scale
+
+
+def test_gemm_full_all_ones_closed_form(orc):
+    M, N, K = 3, 8, 512
+    _, qa = orc.quantize(torch.ones(M, K, dtype=torch.bfloat16))
+    _, qb = orc.quantize(torch.ones(N, K, dtype=torch.bfloat16))
+    g = np.float64(np.float32(1.0) / np.float32(2688.0))
+    want = K * (2688.0 * g) ** 2
+    y = orc.gemm_full(qa, qb)
+    assert np.all(np.abs(y - want) <= K * 2.0 ** -52 * want)
+
+
+def test_bf16_from_f64_rounds_once(orc):
+    """Direct fp64 -> BF16 rounding (to nearest, ties to even) against the oracle's FP32 -> BF16
+    on values that are exact in FP32 (one rounding either way), and on cases where rounding
+    through FP32 first would round twice."""
+    rng = np.random.default_rng(5)
+    bits = rng.integers(0x00800000, 0x7F000000, 200_000, dtype=np.uint64).astype(np.uint32)
+    f = bits.view(np.float32)
+    f = np.concatenate([f, -f, np.float32([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 3.0, 448.0])])
+    assert np.array_equal(orc.bf16_from_f64(f.astype(np.float64)), orc.bf16_from_float_array(f))
+    # 1 + 2^-8 is a tie between 1 (0x3F80, even) and 1 + 2^-7 (0x3F81): the even one
+    assert orc.bf16_from_f64(1.0 + 2.0 ** -8) == 0x3F80
+    assert orc.bf16_from_f64(1.0 + 3 * 2.0 ** -8) == 0x3F82
+    # just above the tie: BF16 rounds up; through FP32 the 2^-30 would vanish first (-> 0x3F80)
+    x = 1.0 + 2.0 ** -8 + 2.0 ** -30
+    assert orc.bf16_from_f64(x) == 0x3F81
+    assert orc.bf16_from_float(np.float32(x)) == 0x3F80
+    assert orc.bf16_from_f64(-x) == 0xBF81
+    assert orc.bf16_from_f64(-(1.0 + 2.0 ** -8)) == 0xBF80

@@ -1,7 +1,7 @@
 """nvfp4_quantize_noalloc: the quantizer for callers that cannot allocate (engine plugin hooks,
 embedded host programs that hand over only their input and output buffers).  It must give the
-same bytes as nvfp4_quantize, which takes a caller-provided workspace, on consecutive calls that
-share its static scratch array.  Called here directly through the C ABI.
+same bytes as nvfp4_quantize, which takes a caller-provided workspace, and as the CPU oracle, on
+consecutive calls that share its static scratch array.  Called here directly through the C ABI.
 
 This file is collected last on purpose; it passes both alone in a fresh process and after the
 rest of the suite."""
@@ -12,6 +12,7 @@ import torch
 
 import bit_kv_cache_24_b200 as nv
 from bit_kv_cache_24_b200 import synth
+from tests.parity_util import assert_quantized_equal
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +34,7 @@ def _same(a, b):
     assert torch.equal(a.g, b.g)
 
 
-def test_noalloc_matches_workspace_quantizer_on_consecutive_calls():
+def test_noalloc_matches_workspace_quantizer_on_consecutive_calls(orc):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     x1 = synth.ragged(21, 4680, 3072, "lognormal").cuda()          # large: fills many scratch slots
     x2 = synth.ragged(22, 130, 96, "outliers").cuda()              # small: fewer slots
@@ -47,6 +48,9 @@ def test_noalloc_matches_workspace_quantizer_on_consecutive_calls():
     third = _noalloc(x1, nv.ROWWISE, nv.SF_MMA, status)
     torch.cuda.synchronize()
     _same(third, first)
+    # the bytes themselves against the CPU oracle
+    assert_quantized_equal(orc, first, orc.quantize(x1.cpu())[1], "no-alloc row-wise")
+    assert_quantized_equal(orc, second, orc.quantize(x2.cpu(), colwise=True)[1], "no-alloc column-wise")
 
 
 def test_noalloc_rejects_bad_arguments_without_launching():
@@ -56,4 +60,7 @@ def test_noalloc_rejects_bad_arguments_without_launching():
     assert nv.lib().nvfp4_quantize_noalloc(None, 16, 32, 32, nv.ROWWISE, ctypes.byref(st), None, None) == \
         nv.NVFP4_ERR_INVALID_ARG
     assert nv.lib().nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), 16, 32, 32, nv.COLWISE,
+                                           ctypes.byref(st), None, None) == nv.NVFP4_ERR_INVALID_ARG
+    # both layouts in one call are not offered here (one output tensor)
+    assert nv.lib().nvfp4_quantize_noalloc(ctypes.c_void_p(x.data_ptr()), 16, 32, 32, nv.ROWCOL,
                                            ctypes.byref(st), None, None) == nv.NVFP4_ERR_INVALID_ARG
