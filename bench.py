@@ -327,9 +327,9 @@ class QKVStep:
         self.side_ops = {"w_quantize"}                    # on the side stream, overlapping the others
         self.launches = 0                                 # kernels launched by step() so far
         # kernels per step: W amax + scale record + row pass; A amax + record + row + column pass;
-        # GEMM + the column-group amax finish; K/V scale record + row pass (both tensors per
-        # launch; their amax comes from the GEMM epilogue); dequant
-        self.launches_per_step = 3 + 4 + 2 + 2 + 1
+        # GEMM + the column-group amax finish; the K/V row pass (both tensors per launch; their
+        # amax comes from the GEMM epilogue and the pass builds its own scale record); dequant
+        self.launches_per_step = 3 + 4 + 2 + 1 + 1
 
     def step(self, i, events=None, A=None, Y=None):
         """One step.  W's quantization is independent of the rest, so it runs on a side stream as
@@ -824,7 +824,7 @@ def run_appends(args, rank, local_rank, world):
                                "of 30 layers", "global_batch": M_TOK * world, "seq_len": M_TOK,
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs rotate over 6 layers' K/V (345 MB) > 126 MB L2"},
-        "gpu_launches": 3 * LAYERS * 2 * K,
+        "gpu_launches": 3 * LAYERS * 2 * K,                 # amax, record, row pass per layer; graph + eager
         "eager": {"ms_per_step": round(eager_s * 1e3 / K, 4),
                   "value": round(APPEND_BYTES * LAYERS * K / eager_s / 1e9, 1), "unit": "GB/s"},
         "roofline": {"kernel": "kv_quant_append (amax, scale record, row pass)", "bound": "hbm",

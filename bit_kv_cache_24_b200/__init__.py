@@ -21,7 +21,9 @@ import re
 import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+# NVFP4_LIB selects another build of the same library (e.g. the bounds-checked debug build,
+# libnvfp4_checked.so); the default is the in-tree release build.
+LIB_PATH = os.environ.get("NVFP4_LIB") or os.path.join(HERE, "libnvfp4.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
 NVFP4_OK, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_UNSUPPORTED = 0, 1, 2

@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
 
 }  // namespace
 
-cudaError_t launch_kv_attention(const AttnJob &j, cudaStream_t s) {
+cudaError_t launch_kv_attention(const AttnJob &j, int32_t *status, cudaStream_t s) {
+    (void)status;                                         // this kernel never waits
     if (j.tq <= 0) return cudaSuccess;
     static std::atomic<bool> attr_set[64];               // per device; a repeated set is harmless
     int dev = 0;

@@ -27,7 +27,8 @@ struct AttnJob {
     float scale_log2;                   // softmax scale * log2(e)
 };
 
-// head_dim is 128 (checked by the caller).
-cudaError_t launch_kv_attention(const AttnJob &j, cudaStream_t s);
+// head_dim is 128 (checked by the caller).  status: the optional device status word (a bounded
+// wait that gives up writes NVFP4_ERR_TIMEOUT there).
+cudaError_t launch_kv_attention(const AttnJob &j, int32_t *status, cudaStream_t s);
 
 }  // namespace nvfp4

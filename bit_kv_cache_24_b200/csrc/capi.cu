@@ -242,8 +242,17 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
     rj.job[0].g_out[0] = row_out ? row_out->g : nullptr;
     rj.job[0].g_out[1] = col_out ? col_out->g : nullptr;
     cudaError_t e = cudaSuccess;
-    if (!amax_in) e = launch_amax(jobs, dev_status, nullptr, s);
-    if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+    if (amax_in) {
+        // one launch per layout: the quantize passes build the scale record from amax_in
+        // themselves; the first pass reports g (both outputs) and a non-finite amax
+        j.amax_in = amax_in;
+        j.status = dev_status;
+        j.g_out[0] = row_out ? row_out->g : col_out->g;
+        j.g_out[1] = row_out && col_out ? col_out->g : nullptr;
+    } else {
+        e = launch_amax(jobs, dev_status, nullptr, s);
+        if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+    }
     if (e == cudaSuccess && row_out) {
         j.codes = row_out->codes;
         j.pitch = codes_pitch(K);
@@ -253,6 +262,10 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
     }
     if (e == cudaSuccess && col_out) {
         RowJob jc = j;
+        if (row_out) {                                    // the row pass reported already
+            jc.g_out[0] = jc.g_out[1] = nullptr;
+            jc.status = nullptr;
+        }
         jc.codes = col_out->codes;
         jc.pitch = codes_pitch(M);
         jc.sf = col_out->sf;
@@ -401,9 +414,17 @@ nvfp4_status kv_quant_append_amax(nvfp4_kv_cache *cache, int32_t layer, int32_t 
         rj.job[i].rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
         rj.job[i].g_out[0] = (i == 0 ? cache->g_k : cache->g_v) + slot_index;
         rj.job[i].g_out[1] = nullptr;
+        if (amax_kv) {                                    // one launch: the row pass builds the record
+            j.amax_in = amax_kv + i;
+            j.g_out[0] = rj.job[i].g_out[0];
+            j.status = dev_status;
+        }
     }
-    cudaError_t e = amax_kv ? cudaSuccess : launch_amax(jobs, dev_status, nullptr, s);
-    if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+    cudaError_t e = cudaSuccess;
+    if (!amax_kv) {
+        e = launch_amax(jobs, dev_status, nullptr, s);
+        if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+    }
     if (e == cudaSuccess) e = launch_quantize_rows(jobs, s);
     if (e != cudaSuccess) return cuda_fail(e, "kv_quant_append");
     cache->len[slot_index] = (int32_t)ntok;
@@ -452,7 +473,6 @@ nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, const int32_
 nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, const int32_t *slots, int32_t nslots,
                           const void *q_bf16, int64_t tq, int64_t ldq, float scale, void *o_bf16, int64_t ldo,
                           int32_t *dev_status, nvfp4_stream stream) {
-    (void)dev_status;                                     // no data-dependent error exists
     if (!kv_ok(cache) || !slots || tq < 0 || (tq > 0 && (!q_bf16 || !o_bf16)) || !std::isfinite(scale))
         return NVFP4_ERR_INVALID_ARG;
     if (layer < 0 || layer >= cache->layers || nslots <= 0 || nslots > kMaxDequantSlots) return NVFP4_ERR_INVALID_ARG;
@@ -495,7 +515,7 @@ nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, const int3
     j.o = static_cast<uint16_t *>(o_bf16);
     j.ldo = ldo;
     j.scale_log2 = (float)((double)scale * 1.4426950408889634);   // log2(e)
-    cudaError_t e = launch_kv_attention(j, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_kv_attention(j, dev_status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "kv_attention");
 }
 

@@ -168,6 +168,42 @@ struct SmemRecord {
     uint32_t ok;
 };
 
+// The record's entries from g (one definition for the record kernel and for the quantize passes
+// that build their record themselves from a given amax): r_tab[sf] = RN(1 / RN(e4m3(sf) * g)),
+// 0 where that product is 0; den = RN(g * 6); inv_den = RN(1 / den), or 0 when den < 2^-125 (the
+// scale quotient then divides).
+__device__ __forceinline__ float record_r_entry(uint32_t sf, float g) {
+    const float d = __fmul_rn(e4m3_to_f32(sf), g);
+    return (d == 0.0f) ? 0.0f : __frcp_rn(d);
+}
+__device__ __forceinline__ float record_den(float g) { return __fmul_rn(g, kE2M1Max); }
+__device__ __forceinline__ float record_inv_den(float den) { return den >= 0x1p-125f ? __frcp_rn(den) : 0.0f; }
+
+// A quantize pass whose amax is given builds the record in shared memory itself (threads
+// 0..128 of the CTA; a barrier must follow).  The CTA with `report` set also writes g to the
+// nullable g_out pointers and, for a non-finite amax, NVFP4_ERR_NONFINITE to the status word
+// (the record's ok flag is then 0 and the pass writes nothing), as the record kernel does.
+__device__ __forceinline__ void build_record(float amax, SmemRecord &s, bool report, float *g_out0, float *g_out1,
+                                             int32_t *status) {
+    const bool finite = isfinite(amax);
+    const float g = global_scale(amax);
+    if (threadIdx.x < 128) s.r_tab[threadIdx.x] = record_r_entry(threadIdx.x, g);
+    if (threadIdx.x == 128) {
+        const float den = record_den(g);
+        s.den = den;
+        s.inv_den = record_inv_den(den);
+        s.ok = finite ? 1u : 0u;
+        if (report) {
+            if (!finite) {
+                set_status(status, NVFP4_ERR_NONFINITE);
+            } else {
+                if (g_out0) *g_out0 = g;
+                if (g_out1) *g_out1 = g;
+            }
+        }
+    }
+}
+
 // ---- the 16-block step --------------------------------------------------------------------------
 //
 // sf = e4m3(RN(b / den)).  The quotient comes from q0 = RN(b * y), y = RN(1/den), corrected once:

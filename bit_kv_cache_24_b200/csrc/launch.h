@@ -33,7 +33,13 @@ struct RowJob {
     uint8_t *sf;
     int32_t sf_layout;      // 0 linear [rows][ceil(cols/16)], 1 tensor-core layout
     uint32_t *partial;      // [kMaxPartials] partial maxima (BF16 magnitude bits), amax pass
-    const ScaleRecord *rec; // read by the quantize passes
+    const ScaleRecord *rec; // read by the quantize passes (unless amax_in is set)
+    // Given amax (device float, nullable): the quantize pass builds its scale record itself
+    // (no record kernel) and its first CTA writes g to g_out[] (nullable) or, for a non-finite
+    // amax, NVFP4_ERR_NONFINITE to status.
+    const float *amax_in;
+    float *g_out[2];
+    int32_t *status;
 };
 
 struct RowJobs {

@@ -251,15 +251,12 @@ __global__ void __launch_bounds__(kThreads) scale_record_kernel(const __grid_con
         return;
     }
     const float g = global_scale(amax);
-    const float den = __fmul_rn(g, kE2M1Max);
-    if (threadIdx.x < 128) {
-        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
-        rec->r_tab[threadIdx.x] = (d == 0.0f) ? 0.0f : __frcp_rn(d);
-    }
+    const float den = record_den(g);
+    if (threadIdx.x < 128) rec->r_tab[threadIdx.x] = record_r_entry(threadIdx.x, g);
     if (threadIdx.x == 128) {
         rec->g = g;
         rec->den = den;
-        rec->inv_den = den >= 0x1p-125f ? __frcp_rn(den) : 0.0f;
+        rec->inv_den = record_inv_den(den);
         rec->ok = 1;
         if (j.g_out[0]) *j.g_out[0] = g;
         if (j.g_out[1]) *j.g_out[1] = g;
@@ -307,7 +304,10 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_co
             for (int i = 0; i < 8; ++i) w[b][i] = 0;
         }
     }
-    load_record(j.rec, rec);
+    if (j.amax_in)
+        build_record(*j.amax_in, rec, blockIdx.x == 0, j.g_out[0], j.g_out[1], j.status);
+    else
+        load_record(j.rec, rec);
     __syncthreads();
     if (!active || !rec.ok) return;
 
@@ -382,7 +382,11 @@ __device__ __forceinline__ void cols_body(const RowJob &j, SmemRecord &rec) {
         }
         w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
     }
-    load_record<kConcurrent>(j.rec, rec);
+    if (j.amax_in)   // concurrent: complete before the row pass started, read through L2
+        build_record(kConcurrent ? __uint_as_float(ldg_cg_u32(j.amax_in)) : *j.amax_in, rec, blockIdx.x == 0,
+                     j.g_out[0], j.g_out[1], j.status);
+    else
+        load_record<kConcurrent>(j.rec, rec);
     __syncthreads();
     if (!active || !rec.ok || kc >= kc_total || mb >= mb_total) return;
 

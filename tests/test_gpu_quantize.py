@@ -142,3 +142,46 @@ def test_repeated_calls_share_workspace(orc):
     for x, g in zip(xs, outs):
         _, o = orc.quantize(x)
         assert_quantized_equal(orc, g, o, "shared ws")
+
+
+@pytest.mark.parametrize("rows,cols,kind", [(37, 48, "outliers"), (300, 96, "wide"), (4680, 3072, "lognormal")])
+@pytest.mark.parametrize("layout", [nv.SF_LINEAR, nv.SF_MMA])
+def test_amax_given_builds_its_record_in_the_pass(orc, rows, cols, kind, layout):
+    """With amax_in the quantize passes build the per-tensor scale record themselves (one launch
+    per layout, no record kernel): row-wise, column-wise and both-layouts outputs and g equal the
+    oracle's quantization with the same amax, byte for byte."""
+    x = synth.ragged(rows * 3 + cols, rows, cols, kind)
+    xg = x.cuda()
+    amax = nv.nvfp4_amax(xg)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    gr = nv.nvfp4_quantize(xg, nv.ROWWISE, amax_in=amax, sf_layout=layout, status=st)
+    gc = nv.nvfp4_quantize(xg, nv.COLWISE, amax_in=amax, sf_layout=layout, status=st)
+    br, bc = nv.nvfp4_quantize(xg, nv.ROWCOL, amax_in=amax, sf_layout=layout, status=st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    a = np.float32(amax.item())
+    _, orow = orc.quantize(x, amax_in=a)
+    _, ocol = orc.quantize(x, colwise=True, amax_in=a)
+    for got, want, label in ((gr, orow, "row"), (gc, ocol, "col"), (br, orow, "rowcol-row"), (bc, ocol, "rowcol-col")):
+        assert_quantized_equal(orc, got, want, f"amax given {label} {rows}x{cols}")
+
+
+@pytest.mark.parametrize("direction", [nv.ROWWISE, nv.COLWISE, nv.ROWCOL])
+def test_nonfinite_amax_in_sets_status_and_writes_nothing(direction):
+    x = synth.ragged(9, 64, 96, "normal").cuda()
+    for bad in (float("inf"), float("nan")):
+        amax = torch.tensor([bad], dtype=torch.float32, device="cuda")
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        outs = nv.nvfp4_quantize(x, direction, amax_in=amax, status=st)
+        outs = outs if isinstance(outs, tuple) else (outs,)
+        for q in outs:
+            q.codes.fill_(0xAB)
+            q.sf.fill_(0xCD)
+            q.g.fill_(-1.0)
+        torch.cuda.synchronize()
+        nv.nvfp4_quantize(x, direction, amax_in=amax, status=st,
+                          out=outs if direction == nv.ROWCOL else outs[0])
+        torch.cuda.synchronize()
+        assert st.item() == nv.NVFP4_ERR_NONFINITE
+        for q in outs:
+            assert bool((q.codes == 0xAB).all()) and bool((q.sf == 0xCD).all()) and q.g.item() == -1.0
