@@ -23,6 +23,13 @@
 //   warps 4-11  epilogue (both CTAs): two warps per tensor-memory lane quarter, 128 columns each;
 //               a warp drains its columns to registers and releases tensor memory before the
 //               scaling, bias/residual add, rounding and stores, which overlap the next tile.
+//               BF16 output leaves through shared memory: per 32 x 32 chunk a warp writes its
+//               rows into a 64-byte-swizzled staging buffer (two per warp) and one lane issues a
+//               TMA tensor store, so every global write is a full line (per-lane 16-byte row
+//               stores to 32 different rows ran the epilogue at ~1.3 TB/s and bounded the GEMM
+//               on the short-K shapes).  FP32 output (accuracy checks) keeps direct stores.
+// Tile order: M-fastest, or N-fastest when A is the larger operand (then a few A stripes are
+// live at a time and all of B stays in L2, instead of every A stripe being re-read per N tile).
 // Tensor memory per CTA: accumulator columns [0, 256), scale buffers per stage after it.
 // Scale tiles are read through 2-D tensor maps over the 512-byte atoms (viewed as uint64), so
 // atom rows past M or N are zero-filled by TMA like the code tiles.
@@ -53,7 +60,10 @@ constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_SFA = OFF_B + STAGES * B_STAGE;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_STAGE;
-constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_STAGE;
+constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_STAGE;   // output staging, 1024-aligned
+constexpr int EPI_BUF = 2048;                           // one warp's 32 rows x 32 BF16 columns
+constexpr int OFF_BAR = OFF_EPI + 8 * 2 * EPI_BUF;      // two buffers per epilogue warp
+static_assert(OFF_EPI % 1024 == 0, "staging alignment (64-byte swizzle period)");
 constexpr int NUM_BARS = 3 * STAGES + 3;            // full[], empty[], sf_full[], tmem_full, tmem_empty, drain
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
@@ -162,8 +172,15 @@ __device__ __forceinline__ void stg_v4(void *p, uint4 v) {
 }
 
 struct Maps {
-    CUtensorMap a, b, sfa, sfb;
+    CUtensorMap a, b, sfa, sfb, y;
+    int y_tma;      // BF16 output through the y map (else direct stores)
+    int n_fast;     // tile order: N index fastest
 };
+
+__device__ __forceinline__ void sts_v4(uint32_t saddr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" :: "r"(saddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__ GemmArgs args) {
@@ -242,7 +259,7 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
         uint32_t stage = 0, phase = 0, used = 0, last_parity = 0;
         bool ok = true;
         for (int t = cluster; ok && t < num_tiles; t += nclusters) {
-            const int mb = t % mt, nb = t / mt;
+            const int mb = maps.n_fast ? t / nt : t % mt, nb = maps.n_fast ? t % nt : t / mt;
             for (int kt = 0; kt < nkt; ++kt) {
                 if (!warp_wait(bar_empty + 8 * stage, phase ^ 1)) {
                     ok = false;
@@ -338,10 +355,13 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
         const bool quant = args.q_rec && qrec.ok;
         const int64_t q_rows = args.q_sf_layout ? 128 * ceil_div(M, 128) : M;
         uint32_t acc_phase = 0;
+        const bool y_tma = maps.y_tma != 0;
+        uint32_t nstores = 0;                             // TMA stores issued by lane 0 of this warp
+        const uint32_t sbuf0 = base + OFF_EPI + (uint32_t)(warp - EPI_WARP0) * 2 * EPI_BUF;
         for (int t = cluster; t < num_tiles; t += nclusters) {
             if (!warp_wait(bar_tmem_full, acc_phase)) break;
             tc_fence_after();
-            const int mb = t % mt, nb = t / mt;
+            const int mb = maps.n_fast ? t / nt : t % mt, nb = maps.n_fast ? t % nt : t / mt;
             const int64_t m = (int64_t)mb * BM + (int64_t)rank * BM_CTA + q * 32 + lane;
             const bool row_ok = m < M;
             const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16) + ACC_COL + half * 128;
@@ -359,6 +379,60 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int64_t n0 = (int64_t)nb * BN + half * 128 + c * 32;
+                if (y_tma) {
+                    const int ym = mb * BM + (int)rank * BM_CTA + q * 32;   // the warp's first row
+                    if (n0 >= N) continue;                                    // warp-uniform
+                    if (ym >= M) {                                            // warp-uniform: no live row
+                        if (quant && m < q_rows) store_sf_pair(args, m, n0 >> 4, 0u);   // scale padding rows
+                        continue;
+                    }
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(alpha, __uint_as_float(r[c][i]));
+                    const uint16_t *addsrc = args.bias ? args.bias + n0
+                                                       : (args.resid && row_ok ? args.resid + m * args.ldy + n0 : nullptr);
+                    if (addsrc) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            if (n0 + 8 * g >= N) break;
+                            const uint4 b = ldg_v4(addsrc + 8 * g);
+                            const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                v[8 * g + 2 * i] = __fadd_rn(v[8 * g + 2 * i], bf16_lo(bw[i]));
+                                v[8 * g + 2 * i + 1] = __fadd_rn(v[8 * g + 2 * i + 1], bf16_hi(bw[i]));
+                            }
+                        }
+                    }
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) w[i] = bf16x2(v[2 * i], v[2 * i + 1]);
+                    const uint32_t sbuf = sbuf0 + (nstores & 1) * EPI_BUF;
+                    // the store issued from this buffer two chunks ago must have finished reading it
+                    if (lane == 0 && nstores >= 2) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+                    __syncwarp();
+                    // lane = row: 64-byte rows, 16-byte chunk g at (g ^ (row / 2) % 4) (SWIZZLE_64B);
+                    // rows past M are written here but clipped by the store
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        sts_v4(sbuf + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4),
+                               make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]));
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) {
+                        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                                     :: "l"(&maps.y), "r"((int)n0), "r"(ym), "r"(sbuf) : "memory");
+                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    }
+                    ++nstores;
+                    if (row_ok) {
+                        if (quant) emit_nvfp4_chunk(args, qrec, m, n0, w);
+                        if (args.cam_partial) cam = max(cam, max(absmax_bits16(w), absmax_bits16(w + 8)));
+                    } else if (quant && m < q_rows) {
+                        store_sf_pair(args, m, n0 >> 4, 0u);
+                    }
+                    continue;
+                }
                 if (!row_ok || n0 >= N) {
                     if (quant && n0 < N && m < q_rows) store_sf_pair(args, m, n0 >> 4, 0u);   // scale padding rows
                     continue;
@@ -414,6 +488,9 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
             }
             acc_phase ^= 1;
         }
+        // the TMA stores must have read the staging buffers and written Y before the CTA exits
+        if (lane == 0 && nstores > 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -474,6 +551,14 @@ cudaError_t launch_gemm_2sm(const GemmArgs &args, cudaStream_t s) {
         encode_2d(&maps.sfb, CU_TENSOR_MAP_DATA_TYPE_UINT64, 8, args.b_sf, ksteps * 64, ceil_div(args.N, 128),
                   ksteps * 512, 256, 2, CU_TENSOR_MAP_SWIZZLE_NONE);
     if (!ok) return cudaErrorInvalidValue;
+    maps.y_tma = 0;
+    if (args.y && !args.y_f32) {      // BF16 Y: 32 x 32 boxes, 64-byte swizzle (row stride ldy % 8 == 0)
+        if (!encode_2d(&maps.y, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, args.y, args.N, args.M, args.ldy * 2, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
+        maps.y_tma = 1;
+    }
+    maps.n_fast = args.M * args.a_pitch > args.N * args.b_pitch ? 1 : 0;
     const int64_t tiles = ceil_div(args.M, BM) * ceil_div(args.N, BN);
     int clusters = num_sms() / 2;
     if (tiles < clusters) clusters = (int)tiles;
