@@ -27,7 +27,7 @@ LIB_PATH = os.environ.get("NVFP4_LIB") or os.path.join(HERE, "libnvfp4.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "nvfp4.h")
 
 NVFP4_OK, NVFP4_ERR_INVALID_ARG, NVFP4_ERR_UNSUPPORTED = 0, 1, 2
-NVFP4_ERR_NONFINITE, NVFP4_ERR_TIMEOUT, NVFP4_ERR_CUDA = 3, 4, 5
+NVFP4_ERR_NONFINITE, NVFP4_ERR_TIMEOUT, NVFP4_ERR_CUDA, NVFP4_ERR_OUT_OF_BOUNDS = 3, 4, 5, 6
 ROWWISE, COLWISE, ROWCOL = 0, 1, 2
 SF_LINEAR, SF_MMA = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
@@ -69,6 +69,7 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         sig = {
             "nvfp4_version": (_I32, []),
+            "nvfp4_checked_build": (_I32, []),
             "nvfp4_status_string": (ctypes.c_char_p, [_I32]),
             "nvfp4_last_error": (ctypes.c_char_p, []),
             "nvfp4_codes_pitch": (_I64, [_I64]),
@@ -95,6 +96,7 @@ def lib():
                                     ctypes.c_float, _P, _I64, _P, _P]),
             "nvfp4_encode_elements": (_I32, [_P, _I64, _P, _P, _P]),
             "nvfp4_selftest_wait_timeout": (_I32, [_P, _I64, _P]),
+            "nvfp4_selftest_bounds": (_I32, [_P, _I64, _I64, _P, _P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -123,6 +125,44 @@ def _stream(stream):
 
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+_checked = None
+_checked_status = {}      # device index -> int32 status word of the binding (checked build only)
+
+
+def checked_build() -> bool:
+    """True when the loaded library is the bounds-checked debug build (NVFP4_LIB selects it)."""
+    global _checked
+    if _checked is None:
+        _checked = bool(lib().nvfp4_checked_build())
+    return _checked
+
+
+def _status(status):
+    """The caller's status word; in the checked build, when the caller passes none, a per-device
+    word of the binding's own, which checked_status() reads back."""
+    if status is not None or not checked_build():
+        return _ptr(status)
+    dev = torch.cuda.current_device()
+    t = _checked_status.get(dev)
+    if t is None:
+        t = _checked_status[dev] = torch.zeros(1, dtype=torch.int32, device=torch.device("cuda", dev))
+    return _ptr(t)
+
+
+def checked_status(reset: bool = True) -> int:
+    """Checked build: the first nonzero code the kernels wrote to the binding's own status words
+    (calls made without a status argument), 0 if none; synchronizes each device first."""
+    code = 0
+    for dev, t in _checked_status.items():
+        with torch.cuda.device(dev):
+            torch.cuda.synchronize()
+            v = int(t.item())
+            if reset:
+                t.zero_()
+        code = code or v
+    return code
 
 
 def _ws(nbytes, device):
@@ -163,7 +203,7 @@ def nvfp4_amax(x, out=None, ws=None, status=None, stream=None):
     out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
     nws = L.nvfp4_quantize_workspace(M, K)
     ws = _ws(nws, x.device) if ws is None else ws
-    _check("nvfp4_amax", L.nvfp4_amax(_ptr(x), M, K, x.stride(0), _ptr(out), _ptr(ws), ws.numel(), _ptr(status),
+    _check("nvfp4_amax", L.nvfp4_amax(_ptr(x), M, K, x.stride(0), _ptr(out), _ptr(ws), ws.numel(), _status(status),
                                       _stream(stream)))
     return out
 
@@ -186,7 +226,7 @@ def nvfp4_quantize(x, dir=ROWWISE, amax_in=None, out=None, sf_layout=SF_MMA, ws=
     outs = out if isinstance(out, tuple) else (out,)
     st = (_Tensor * len(outs))(*[o.struct() for o in outs])
     _check("nvfp4_quantize", L.nvfp4_quantize(_ptr(x), M, K, x.stride(0), dir, _ptr(amax_in), st,
-                                              _ptr(ws), 0 if ws is None else ws.numel(), _ptr(status),
+                                              _ptr(ws), 0 if ws is None else ws.numel(), _status(status),
                                               _stream(stream)))
     return out
 
@@ -201,7 +241,7 @@ def nvfp4_gemm(A: QTensor, B: QTensor, bias=None, resid=None, out=None, out_dtyp
                           device=A.codes.device)
     sa, sb = A.struct(), B.struct()
     _check("nvfp4_gemm", L.nvfp4_gemm(ctypes.byref(sa), ctypes.byref(sb), _ptr(bias), _ptr(resid), _ptr(out),
-                                      out.stride(0), out_dtype, _ptr(status), _stream(stream)))
+                                      out.stride(0), out_dtype, _status(status), _stream(stream)))
     return out
 
 
@@ -221,7 +261,7 @@ def nvfp4_gemm_quant_out(A: QTensor, B: QTensor, amax_in, bias=None, resid=None,
     sa, sb, sq = A.struct(), B.struct(), q_out.struct()
     _check("nvfp4_gemm_quant_out", L.nvfp4_gemm_quant_out(ctypes.byref(sa), ctypes.byref(sb), _ptr(bias), _ptr(resid),
                                                           _ptr(out), ldy, _ptr(amax_in), ctypes.byref(sq), _ptr(ws),
-                                                          ws.numel(), _ptr(status), _stream(stream)))
+                                                          ws.numel(), _status(status), _stream(stream)))
     return out, q_out
 
 
@@ -241,7 +281,7 @@ def nvfp4_gemm_colamax(A: QTensor, B: QTensor, group_cols, bias=None, resid=None
     sa, sb = A.struct(), B.struct()
     _check("nvfp4_gemm_colamax", L.nvfp4_gemm_colamax(ctypes.byref(sa), ctypes.byref(sb), _ptr(bias), _ptr(resid),
                                                       _ptr(out), out.stride(0), group_cols, _ptr(amax_out), _ptr(ws),
-                                                      ws.numel(), _ptr(status), _stream(stream)))
+                                                      ws.numel(), _status(status), _stream(stream)))
     return out, amax_out
 
 
@@ -288,11 +328,11 @@ def kv_quant_append(cache: KVCache, layer, slot, k, v, status=None, stream=None,
     if amax_kv is None:
         _check("kv_quant_append", lib().kv_quant_append(ctypes.byref(cache._c), layer, slot, _ptr(k2), _ptr(v2),
                                                         k2.shape[0], k2.stride(0), _ptr(cache.ws), cache.ws.numel(),
-                                                        _ptr(status), _stream(stream)))
+                                                        _status(status), _stream(stream)))
     else:
         _check("kv_quant_append_amax", lib().kv_quant_append_amax(ctypes.byref(cache._c), layer, slot, _ptr(k2),
                                                                   _ptr(v2), k2.shape[0], k2.stride(0), _ptr(amax_kv),
-                                                                  _ptr(cache.ws), cache.ws.numel(), _ptr(status),
+                                                                  _ptr(cache.ws), cache.ws.numel(), _status(status),
                                                                   _stream(stream)))
 
 
@@ -306,7 +346,7 @@ def kv_dequant(cache: KVCache, layer, slots, k_out=None, v_out=None, status=None
     v_out = torch.empty(shape, dtype=torch.bfloat16, device=dev) if v_out is None else v_out
     arr = (_I32 * len(slots))(*slots)
     _check("kv_dequant", lib().kv_dequant(ctypes.byref(cache._c), layer, arr, len(slots), _ptr(k_out), _ptr(v_out),
-                                          _ptr(status), _stream(stream)))
+                                          _status(status), _stream(stream)))
     return k_out, v_out
 
 
@@ -334,7 +374,7 @@ def kv_attention(cache: KVCache, layer, slots, q, scale, out=None, status=None, 
     slots = [int(s) for s in slots]
     arr = (_I32 * len(slots))(*slots)
     _check("kv_attention", lib().kv_attention(ctypes.byref(cache._c), layer, arr, len(slots), _ptr(q), tq, ldq,
-                                              float(scale), _ptr(out), ldo, _ptr(status), _stream(stream)))
+                                              float(scale), _ptr(out), ldo, _status(status), _stream(stream)))
     return out
 
 

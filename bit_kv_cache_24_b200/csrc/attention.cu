@@ -1,28 +1,38 @@
 // attention.cu -- softmax attention of BF16 queries over a window of NVFP4 KV-cache slots, with
-// the restore fused into the K/V tile loads.
+// the restore fused into the kernel's K/V tile loads (the restored BF16 K and V never reach HBM).
 //
 // LongLive-2.0 keeps its KV cache in NVFP4 and restores it with a parallel dequantization kernel
-// before attention, FlashAttention being its attention backend (d9249.github.io review, section
-// "핵심 아이디어 / 구조 / 동작 방식"; yourai.pro report).  Here the restore happens inside the
-// attention kernel: a CTA reads the window's codes and scales (0.5625 B per element) and
-// dequantizes every K/V tile into shared memory, so the BF16 K and V (2 B per element) are
-// neither written to nor read from HBM.
+// before attention (d9249.github.io review, section "핵심 아이디어 / 구조 / 동작 방식"; the arXiv
+// abstract on fugumt.com: NVFP4 KV cache for memory savings).  This kernel computes the same
+// attention without the restored copy:
+//   O[i,h,:] = sum_j softmax_j(scale * q[i,h,:] . k[j,h,:]) v[j,h,:],
+// k and v being exactly the values the restore produces, BF16(FP32(e2m1 * sf) * g).
 //
-// O[i,h,:] = sum_j softmax_j(scale * q[i,h,:] . k[j,h,:]) v[j,h,:] over the window's tokens, with
-// k, v = BF16(FP32(e2m1 * sf) * g), the values the restore kernel produces.  No mask.
+// Structure (sm_100a, tcgen05): a CTA owns 256 queries of one head as two 128-row Q tiles and
+// walks the window in 128-token K/V tiles.  416 threads:
+//   warps 0-3   softmax of Q tile 0: thread = query row = tensor-memory lane
+//   warps 4-7   softmax of Q tile 1 (same lanes, its own tensor-memory columns)
+//   warps 8-11  producer: both Q tiles once, then per K/V tile the restore of one token row of K
+//               and of V into shared memory (two stages), the next tile's raw bytes already in
+//               registers
+//   warp 12     MMA issuer (tcgen05.mma kind::f16, BF16 in, FP32 accumulate in tensor memory):
+//                 S_t = Q_t K_i^T  (A = Q_t, B = K_i: both K-major, 128-byte swizzle, in smem)
+//                 O_t += P_t V_i   (A = P_t in TENSOR memory, B = V_i: MN-major in smem)
+// Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); the
+// softmax writes P_t (BF16 pairs) over the first 64 columns of S_t once it has read S_t.
+// The two Q tiles alternate: while one softmax warpgroup works on tile i, the tensor core runs
+// the other Q tile's S or P.V, and the producer restores tile i + 1.  Per Q tile the order is
+// S(i) -> softmax(i) -> P.V(i) -> S(i + 1); one thread issues all MMAs, whose execution is in
+// issue order, so S(i + 1) overwrites P(i) only after P.V(i) has read it.
 //
-// Design (warp-level BF16 MMA, FlashAttention-2 structure):
-//   - CTA = 128 query rows of one head, 8 warps x 16 rows; Q stays in registers as MMA A
-//     fragments. Each CTA dequantizes its head's whole window once, so more rows per CTA means
-//     less dequantization per FLOP.
-//   - Per 64-token tile, each thread holds the raw bytes of half a token row of K or of V (32
-//     code bytes, 4 scale bytes) fetched one tile ahead. It dequantizes them into a
-//     double-buffered shared-memory tile. Rows are padded to 272 B, so neither the 16-byte
-//     stores nor ldmatrix conflict on banks.
-//   - S = Q K^T runs on mma.sync m16n8k16 with FP32 accumulation. Then an online softmax in
-//     base 2, with the row max and sum combined across the quad by shuffles.
-//   - P is rounded to BF16 for O += P V (V fragments by ldmatrix.trans).
-//   - Tokens past the window's end score -inf. The only waits are __syncthreads.
+// Barriers (all waits time-bounded; a wait that gives up raises the abort flag and writes
+// NVFP4_ERR_TIMEOUT to the status word, and every role leaves its loop):
+//   kv_full[2]   count 128: the producers restored the stage (before tile 0: also both Q tiles)
+//   kv_empty[2]  count 1:   commit after the last MMA that reads the stage (P.V of Q tile 1)
+//   s_full[t]    count 1:   commit after S_t(i) (implies P.V_t(i - 1) done, so O_t is stable)
+//   p_full[t]    count 128: softmax t wrote P_t(i) and rescaled O_t
+//   o_done[t]    count 1:   commit after the last P.V_t
+//   drain        count 1:   every MMA retired (before tensor memory is freed)
 #include <atomic>
 #include <cmath>
 
@@ -33,42 +43,140 @@ namespace nvfp4 {
 
 namespace {
 
-constexpr int kD = 128;                     // head_dim
-constexpr int kBQ = 128;                    // query rows per CTA
-constexpr int kBK = 64;                     // window tokens per tile
-constexpr int kThreads = 256;
-constexpr int kPitch = kD * 2 + 16;         // bytes per shared-memory tile row
-constexpr int kTileBytes = kBK * kPitch;
-constexpr int kSmemBytes = 4 * kTileBytes;  // K and V, two buffers each
+constexpr int kD = 128, kBQ = 128, kBKV = 128;
+constexpr int kQTiles = 2;                         // Q tiles per CTA
+constexpr int kThreads = 416;
+constexpr int kRegion = 128 * 128;                 // bytes: 128 rows x 128 B (one 64-wide d half)
+constexpr int OFF_Q = 0;                           // Q tile t at t * 2 regions
+constexpr int OFF_KV = kQTiles * 2 * kRegion;      // stage s: K at OFF_KV + s * 4R, V at + 2R
+constexpr int KV_STAGE = 4 * kRegion;
+constexpr int OFF_BAR = OFF_KV + 2 * KV_STAGE;
+constexpr int NUM_BARS = 2 + 2 + 2 + 2 + 2 + 1;
+constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+constexpr int kSmemBytes = OFF_MISC + 16 + 1024;
+constexpr uint32_t TMEM_COLS = 512, S_COL = 0, O_COL = 256;
 
-static_assert(kThreads == 4 * kBK, "a thread loads half a token row of K or of V");
-static_assert(kBQ == 16 * (kThreads / 32), "a warp owns 16 query rows");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
 
-// y = BF16(FP32(e2m1 * sf) * g) for the 8 codes of one word: the restore's rounding steps (the
-// e2m1 * sf product is exact in FP32, one rounding by g, one to BF16).
-__device__ __forceinline__ uint4 restore8(uint32_t codes, float sf, float g) {
+// kind::f16 instruction descriptors: F32 accumulate (bit 4), A and B BF16 (bits 7, 10), N >> 3
+// at bit 17, M >> 4 at bit 24; b_major (bit 16) = 1 for the MN-major V operand.
+constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBKV >> 3) << 17) |
+                             ((uint32_t)(kBQ >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(kD >> 3) << 17) |
+                              ((uint32_t)(kBQ >> 4) << 24);
+
+// K-major SW128 shared-memory descriptor (SBO = 1024: 8 rows of 128 B), version 1, layout 2.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// MN-major SW128 descriptor: LBO = distance of the two 64-wide d halves (one region), SBO = 1024
+// (8 token rows of 128 B).
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)(kRegion >> 4) << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+
+// Byte offset of 16-byte chunk c (0..15 along a 256-byte logical row) of row r in a pair of SW128
+// regions (chunks 0-7 in the first region, 8-15 in the second).
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+    return (uint32_t)((c >> 3) * kRegion + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\t"
+                 "@p tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+                 :: "r"(bar) : "memory");
+}
+
+// D (tensor memory) = / += A (shared memory) . B (shared memory)
+__device__ __forceinline__ void tc_mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 :: "r"(d), "l"(a), "l"(b), "r"(idesc), "r"(accum) : "memory");
+}
+
+// D (tensor memory) = / += A (tensor memory) . B (shared memory)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t accum) {
+    asm volatile("{\n\t.reg .pred p, e;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "elect.sync _|e, 0xffffffff;\n\t"
+                 "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+                 :: "r"(d), "r"(a), "l"(b), "r"(idesc), "r"(accum) : "memory");
+}
+
+__device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+                   "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+}
+
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+                 "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+                 "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+                 :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+                    "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+                    "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+                    "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+                 : "memory");
+}
+
+// The block scale byte as an f16 pair (sf, sf) (E4M3 -> f16 is exact).
+__device__ __forceinline__ uint32_t sf_f16x2(uint32_t byte) {
+    uint32_t h2;
+    const uint16_t in = (uint16_t)((byte & 0xFFu) * 0x101u);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+    return h2;
+}
+
+// Eight restored values y = BF16(FP32(e2m1 * sf) * g) from 8 codes packed in one word, the
+// restore's rounding steps: e2m1 * sf is formed in f16 pairs, where it is exact (at most 6
+// significant bits, 2^-10 <= |product| <= 2688), widened to FP32 exactly, multiplied by g in FP32
+// (one rounding, paired) and rounded to BF16.
+__device__ __forceinline__ uint4 restore8(uint32_t codes, uint32_t sfh2, float g) {
     uint32_t h[4];
     e2m1x8_to_f16x2(codes, h);
     uint32_t o[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float lo = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(h[i] & 0xFFFFu))), sf);
-        const float hi = __fmul_rn(__half2float(__ushort_as_half((unsigned short)(h[i] >> 16))), sf);
-        o[i] = bf16x2(__fmul_rn(lo, g), __fmul_rn(hi, g));
+        uint32_t pr;
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(pr) : "r"(h[i]), "r"(sfh2));
+        const float lo = __half2float(__ushort_as_half((unsigned short)(pr & 0xFFFFu)));
+        const float hi = __half2float(__ushort_as_half((unsigned short)(pr >> 16)));
+        unsigned long long d;
+        asm("{\n\t.reg .b64 x, y;\n\t"
+            "mov.b64 x, {%1, %2};\n\t"
+            "mov.b64 y, {%3, %3};\n\t"
+            "mul.rn.f32x2 %0, x, y;\n\t}"
+            : "=l"(d) : "f"(lo), "f"(hi), "f"(g));
+        o[i] = bf16x2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
     }
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 __device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
     uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
     return v;
 }
 
-__device__ __forceinline__ uint32_t ldg_nc_u32(const void *p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+__device__ __forceinline__ uint2 ldg_nc_v2(const void *p) {
+    uint2 v;
+    asm volatile("ld.global.nc.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
     return v;
 }
 
@@ -77,193 +185,363 @@ __device__ __forceinline__ void sts_v4(uint32_t saddr, uint4 v) {
                  : "memory");
 }
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t r[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(saddr) : "memory");
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// (a.x, a.y) * (b, b) + (c, c) and (a.x, a.y) + (b.x, b.y): paired FP32 operations, IEEE RN
+__device__ __forceinline__ float2 fma2(float2 a, float b, float c) {
+    unsigned long long d;
+    asm("{\n\t.reg .b64 x, y, z;\n\t"
+        "mov.b64 x, {%1, %2};\n\t"
+        "mov.b64 y, {%3, %3};\n\t"
+        "mov.b64 z, {%4, %4};\n\t"
+        "fma.rn.f32x2 %0, x, y, z;\n\t}"
+        : "=l"(d) : "f"(a.x), "f"(a.y), "f"(b), "f"(c));
+    return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
 }
 
-__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t saddr, uint32_t r[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(saddr) : "memory");
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    unsigned long long d;
+    asm("{\n\t.reg .b64 x, y;\n\t"
+        "mov.b64 x, {%1, %2};\n\t"
+        "mov.b64 y, {%3, %4};\n\t"
+        "add.rn.f32x2 %0, x, y;\n\t}"
+        : "=l"(d) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
 }
 
-// c += a . b for one 16 x 8 x 16 BF16 tile, FP32 accumulation.
-__device__ __forceinline__ void mma_bf16(float c[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-                 "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-// Raw NVFP4 bytes of half a token row (64 elements) of K or of V, and the slot's g.
-struct Raw {
-    uint4 c[2];
-    uint32_t sf;
-    float g;
-};
+__global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_constant__ AttnJob j,
+                                                                    int32_t *status) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *sbase = smem_raw + (base - raw);
+    const uint32_t bar_kv_full = base + OFF_BAR, bar_kv_empty = bar_kv_full + 16, bar_s_full = bar_kv_empty + 16;
+    const uint32_t bar_p_full = bar_s_full + 16, bar_o_done = bar_p_full + 16, bar_drain = bar_o_done + 16;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sbase + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + OFF_MISC + 4);
+    const int warp = __shfl_sync(0xFFFFFFFFu, (int)(threadIdx.x >> 5), 0);
+    const int lane = threadIdx.x & 31;
+    const int head = blockIdx.y;
+    const int64_t q0 = (int64_t)blockIdx.x * (kQTiles * kBQ);
+    const int ntiles = (int)((j.total_tokens + kBKV - 1) / kBKV);
 
-// Fetch window token `tok` of K (v == 0) or V (v == 1), zeros past the end; `si` is the
-// thread's running slot index (tokens only grow, so it only moves forward).
-__device__ __forceinline__ void fetch(const AttnJob &j, int64_t tok, int &si, int head, int hf, int v, Raw &w) {
-    w.c[0] = w.c[1] = make_uint4(0, 0, 0, 0);
-    w.sf = 0;
-    w.g = 0.0f;
-    if (tok >= j.total_tokens) return;
-    while (si + 1 < j.nslots && tok >= j.slot[si + 1].tok_begin) ++si;
-    const AttnSlot &s = j.slot[si];
-    const int64_t t = tok - s.tok_begin;
-    const uint8_t *codes = v ? s.codes_v : s.codes_k;
-    const int64_t cb = t * j.row_bytes + head * (kD / 2) + hf * 32;
-    w.c[0] = ldg_nc_v4(codes + cb);
-    w.c[1] = ldg_nc_v4(codes + cb + 16);
-    w.sf = ldg_nc_u32((v ? s.sf_v : s.sf_k) + t * j.row_sf + head * (kD / 16) + hf * 4);
-    w.g = *(v ? s.g_v : s.g_k);
-}
-
-// Dequantize one half row (8 words of codes, 4 block scales) into shared memory at `dst`.
-__device__ __forceinline__ void put_half(uint32_t dst, const uint4 c[2], uint32_t sf, float g) {
-    const uint32_t cw[8] = {c[0].x, c[0].y, c[0].z, c[0].w, c[1].x, c[1].y, c[1].z, c[1].w};
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float s = e4m3_to_f32((sf >> (8 * (i >> 1))) & 0xFFu);   // 16-block i/2
-        sts_v4(dst + 16 * i, restore8(cw[i], s, g));
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_kv_full + 8 * i, 128);
+            mbar_init(bar_kv_empty + 8 * i, 1);
+            mbar_init(bar_s_full + 8 * i, 1);
+            mbar_init(bar_p_full + 8 * i, 128);
+            mbar_init(bar_o_done + 8 * i, 1);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbarrier_init();
     }
-}
-
-__global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_constant__ AttnJob j) {
-    extern __shared__ __align__(128) uint8_t smem[];
+    if (warp == 12) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_addr(tmem_slot)), "r"(TMEM_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = __shfl_sync(0xFFFFFFFFu, *tmem_slot, 0);
     griddep_wait();                                       // the cache and q written by earlier kernels
     griddep_launch_dependents();
-    const int head = blockIdx.y;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, tq4 = lane & 3;              // MMA fragment row group, column pair
-    const int64_t r0 = (int64_t)blockIdx.x * kBQ + warp * 16 + g, r1 = r0 + 8;
 
-    // Q A fragments of this warp's 16 rows (rows past tq are zero and not stored)
-    uint32_t qa[kD / 16][4];
-#pragma unroll
-    for (int kk = 0; kk < kD / 16; ++kk) {
-        const int c = head * kD + kk * 16 + tq4 * 2;
-        qa[kk][0] = r0 < j.tq ? *reinterpret_cast<const uint32_t *>(j.q + r0 * j.ldq + c) : 0u;
-        qa[kk][1] = r1 < j.tq ? *reinterpret_cast<const uint32_t *>(j.q + r1 * j.ldq + c) : 0u;
-        qa[kk][2] = r0 < j.tq ? *reinterpret_cast<const uint32_t *>(j.q + r0 * j.ldq + c + 8) : 0u;
-        qa[kk][3] = r1 < j.tq ? *reinterpret_cast<const uint32_t *>(j.q + r1 * j.ldq + c + 8) : 0u;
-    }
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        set_status(status, NVFP4_ERR_TIMEOUT);
+    };
+    // lane 0 of a converged warp waits and broadcasts the outcome, so no warp diverges on it
+    auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        bool ok = true;
+        if (lane == 0) {
+            ok = mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs);
+            if (!ok) give_up();
+        }
+        return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+    };
 
-    float o[kD / 8][4];
+    if (warp >= 8 && warp < 12) {
+        // ------------------------------------------------------------ producer (128 threads)
+        const int t = threadIdx.x - 256;                  // token row of the K/V tile; Q rows t, t + 128
 #pragma unroll
-    for (int n = 0; n < kD / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.0f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;   // rows g and g + 8
-
-    // loader: token row, half of it, K or V
-    const int lr = threadIdx.x & (kBK - 1), hf = (threadIdx.x / kBK) & 1, lv = threadIdx.x / (2 * kBK);
-    const int mi = lane >> 3, mr = lane & 7;              // ldmatrix: matrix, row within it
-    int si = 0;
-    Raw w;
-    fetch(j, lr, si, head, hf, lv, w);
-    const uint32_t sbase = smem_addr(smem);
-    const int64_t ntiles = (j.total_tokens + kBK - 1) / kBK;
-    for (int64_t it = 0; it < ntiles; ++it) {
-        // Buffer it & 1: every warp finished tile it - 2 (which used it) before passing the
-        // barrier of tile it - 1, so it can be overwritten now.
-        const uint32_t kb = sbase + (uint32_t)(it & 1) * 2u * kTileBytes, vb = kb + kTileBytes;
-        put_half((lv ? vb : kb) + lr * kPitch + hf * 128, w.c, w.sf, w.g);
-        if (it + 1 < ntiles) fetch(j, (it + 1) * kBK + lr, si, head, hf, lv, w);
-        __syncthreads();
-
-        // S = Q K^T: 16 rows x 64 tokens per warp
-        float s[kBK / 8][4];
+        for (int qt = 0; qt < kQTiles; ++qt) {
+            const int64_t r = q0 + qt * kBQ + t;
+            const uint16_t *src = j.q + r * j.ldq + head * kD;
+            const uint32_t qb = base + OFF_Q + qt * 2 * kRegion;
 #pragma unroll
-        for (int n = 0; n < kBK / 8; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.0f;
+            for (int c = 0; c < 16; ++c) {
+                const uint4 v = r < j.tq && NVFP4_CHECKED(r * j.ldq + head * kD + 8 * c, 8, j.q_elems, status)
+                                    ? ldg_nc_v4(src + 8 * c) : make_uint4(0, 0, 0, 0);
+                sts_v4(qb + sw_off(t, c), v);
+            }
+        }
+        // the raw NVFP4 bytes of this thread's token row of a tile: loaded before the wait for the
+        // tile's stage, so the loads overlap it
+        struct RawRow {
+            uint4 ck[4], cv[4];
+            uint2 sfk, sfv;
+            float gk, gv;
+            bool live;
+        };
+        int si = 0;
+        auto load_row = [&](int i, RawRow &rr) {
+            const int64_t tok = (int64_t)i * kBKV + t;
+            rr.live = i < ntiles && tok < j.total_tokens;
+            if (!rr.live) return;
+            while (si + 1 < j.nslots && tok >= j.slot[si + 1].tok_begin) ++si;
+            const AttnSlot &s = j.slot[si];
+            const int64_t tt = tok - s.tok_begin;
+            const int64_t cb = tt * j.row_bytes + head * (kD / 2), sb = tt * j.row_sf + head * (kD / 16);
+            // checked build: the token row's codes (64 B) and scales (8 B) inside the slot
+            rr.live = NVFP4_CHECKED(cb, kD / 2, s.ntok * j.row_bytes, status) &&
+                      NVFP4_CHECKED(sb, kD / 16, s.ntok * j.row_sf, status);
+            if (!rr.live) return;
+            rr.gk = *s.g_k;
+            rr.gv = *s.g_v;
+            rr.sfk = ldg_nc_v2(s.sf_k + sb);
+            rr.sfv = ldg_nc_v2(s.sf_v + sb);
 #pragma unroll
-        for (int np = 0; np < kBK / 16; ++np) {
+            for (int q = 0; q < 4; ++q) {
+                rr.ck[q] = ldg_nc_v4(s.codes_k + cb + 16 * q);
+                rr.cv[q] = ldg_nc_v4(s.codes_v + cb + 16 * q);
+            }
+        };
+        bool ok = true;
+        for (int i = 0; ok && i < ntiles; ++i) {
+            const int st = i & 1;
+            RawRow cur;
+            load_row(i, cur);                             // in flight while the stage is awaited
+            if (i >= 2 && !warp_wait(bar_kv_empty + 8 * st, ((i >> 1) - 1) & 1)) { ok = false; break; }
+            const uint32_t kb = base + OFF_KV + st * KV_STAGE, vb = kb + 2 * kRegion;
+            if (cur.live) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {             // 16 B of codes = 32 elements = chunks 4q..4q+3
+                    const uint32_t wk = q < 2 ? cur.sfk.x : cur.sfk.y, wv = q < 2 ? cur.sfv.x : cur.sfv.y;
+                    const uint32_t k0 = sf_f16x2(wk >> (16 * (q & 1))), k1 = sf_f16x2(wk >> (16 * (q & 1) + 8));
+                    const uint32_t v0 = sf_f16x2(wv >> (16 * (q & 1))), v1 = sf_f16x2(wv >> (16 * (q & 1) + 8));
+                    sts_v4(kb + sw_off(t, 4 * q + 0), restore8(cur.ck[q].x, k0, cur.gk));
+                    sts_v4(kb + sw_off(t, 4 * q + 1), restore8(cur.ck[q].y, k0, cur.gk));
+                    sts_v4(kb + sw_off(t, 4 * q + 2), restore8(cur.ck[q].z, k1, cur.gk));
+                    sts_v4(kb + sw_off(t, 4 * q + 3), restore8(cur.ck[q].w, k1, cur.gk));
+                    sts_v4(vb + sw_off(t, 4 * q + 0), restore8(cur.cv[q].x, v0, cur.gv));
+                    sts_v4(vb + sw_off(t, 4 * q + 1), restore8(cur.cv[q].y, v0, cur.gv));
+                    sts_v4(vb + sw_off(t, 4 * q + 2), restore8(cur.cv[q].z, v1, cur.gv));
+                    sts_v4(vb + sw_off(t, 4 * q + 3), restore8(cur.cv[q].w, v1, cur.gv));
+                }
+            } else {                                      // past the window: zero K and V rows
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    sts_v4(kb + sw_off(t, c), make_uint4(0, 0, 0, 0));
+                    sts_v4(vb + sw_off(t, c), make_uint4(0, 0, 0, 0));
+                }
+            }
+            fence_async_smem();                           // generic-proxy writes -> tensor core
+            mbar_arrive(bar_kv_full + 8 * st);
+        }
+    } else if (warp == 12) {
+        // ------------------------------------------------------------ MMA issuer (whole warp)
+        bool ok = true, issued = false;
+        // S_t(i) = Q_t K_i^T into S_t; the stage's K is read by both Q tiles
+        auto issue_s = [&](int qt, int i) {
+            const uint64_t qdesc = kmajor_desc(base + OFF_Q + qt * 2 * kRegion);
+            const uint64_t kdesc = kmajor_desc(base + OFF_KV + (i & 1) * KV_STAGE);
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {
-                uint32_t b[4];
-                ldmatrix_x4(kb + (np * 16 + (mi >> 1) * 8 + mr) * kPitch + (kk * 16 + (mi & 1) * 8) * 2, b);
-                mma_bf16(s[2 * np], qa[kk], b[0], b[1]);
-                mma_bf16(s[2 * np + 1], qa[kk], b[2], b[3]);
+                // K step kk: region kk / 4, 32 bytes per step inside the 128-byte row
+                const uint64_t off = (uint64_t)((kk >> 2) * (kRegion >> 4) + 2 * (kk & 3));
+                tc_mma_ss(tmem + S_COL + 128 * qt, qdesc + off, kdesc + off, kIdescS, kk != 0);
             }
+            tc_commit(bar_s_full + 8 * qt);
+            issued = true;
+        };
+        // O_t += P_t(i) V_i: A = P_t (BF16 pairs in the first 64 columns of S_t), B = V_i
+        auto issue_pv = [&](int qt, int i) {
+            const uint32_t vbase = base + OFF_KV + (i & 1) * KV_STAGE + 2 * kRegion;
+#pragma unroll
+            for (int kt = 0; kt < kBKV / 16; ++kt)
+                tc_mma_ts(tmem + O_COL + 128 * qt, tmem + S_COL + 128 * qt + 8 * kt, mnmajor_desc(vbase + 2048 * kt),
+                          kIdescPV, (i | kt) != 0);
+        };
+        if (ntiles > 0 && warp_wait(bar_kv_full, 0)) {
+            tc_fence_after();
+            issue_s(0, 0);
+            issue_s(1, 0);
+        } else {
+            ok = false;
         }
-
-        // online softmax (base 2): scale, mask the tokens past the window, new row maxima
-        const int64_t t0 = it * kBK;
-        float x0 = -INFINITY, x1 = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < kBK / 8; ++n) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const bool ok = t0 + n * 8 + tq4 * 2 + e < j.total_tokens;
-                s[n][e] = ok ? s[n][e] * j.scale_log2 : -INFINITY;
-                s[n][2 + e] = ok ? s[n][2 + e] * j.scale_log2 : -INFINITY;
-                x0 = fmaxf(x0, s[n][e]);
-                x1 = fmaxf(x1, s[n][2 + e]);
+        for (int i = 0; ok && i < ntiles; ++i) {
+            const bool more = i + 1 < ntiles;
+            // Q tile 0: P.V(i), then S(i + 1) as soon as K(i + 1) is restored
+            if (!warp_wait(bar_p_full, i & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(0, i);
+            if (!more) tc_commit(bar_o_done);
+            if (more) {
+                if (!warp_wait(bar_kv_full + 8 * ((i + 1) & 1), ((i + 1) >> 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                issue_s(0, i + 1);
             }
+            // Q tile 1: P.V(i) frees stage i % 2, then S(i + 1)
+            if (!warp_wait(bar_p_full + 8, i & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(1, i);
+            tc_commit(bar_kv_empty + 8 * (i & 1));
+            if (!more) tc_commit(bar_o_done + 8);
+            if (more) issue_s(1, i + 1);
         }
-        x0 = fmaxf(x0, __shfl_xor_sync(0xFFFFFFFFu, x0, 1));
-        x0 = fmaxf(x0, __shfl_xor_sync(0xFFFFFFFFu, x0, 2));
-        x1 = fmaxf(x1, __shfl_xor_sync(0xFFFFFFFFu, x1, 1));
-        x1 = fmaxf(x1, __shfl_xor_sync(0xFFFFFFFFu, x1, 2));
-        const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-        const float b0 = n0 == -INFINITY ? 0.0f : n0, b1 = n1 == -INFINITY ? 0.0f : n1;   // no inf - inf
-        const float a0 = exp2f(m0 - b0), a1 = exp2f(m1 - b1);
-        m0 = n0;
-        m1 = n1;
-        l0 *= a0;
-        l1 *= a1;
-#pragma unroll
-        for (int n = 0; n < kD / 8; ++n) {
-            o[n][0] *= a0;
-            o[n][1] *= a0;
-            o[n][2] *= a1;
-            o[n][3] *= a1;
+        if (issued) {
+            tc_commit(bar_drain);
+            if (lane == 0 && !mbar_wait_bounded(bar_drain, 0, nullptr, kWaitLimitNs)) give_up();
         }
-
-        // P (BF16) as A fragments: tokens 16kk..16kk+15 come from S tiles 2kk and 2kk + 1
-        uint32_t pa[kBK / 16][4];
+        __syncwarp();
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int qt = warp >> 2;                         // Q tile of this warpgroup
+        const int r = threadIdx.x & 127;                  // query row = tensor-memory lane
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t scol = lane_base + S_COL + 128 * qt, ocol = lane_base + O_COL + 128 * qt;
+        const uint32_t s_full = bar_s_full + 8 * qt, p_full = bar_p_full + 8 * qt;
+        float m = -INFINITY, l = 0.0f;
+        bool ok = true;
+        for (int i = 0; ok && i < ntiles; ++i) {
+            if (!warp_wait(s_full, i & 1)) { ok = false; break; }
+            tc_fence_after();
+            const int64_t t0 = (int64_t)i * kBKV;
+            const bool full = t0 + kBKV <= j.total_tokens;
+            // pass 1: the row maximum of the tile's raw scores (tokens past the window excluded);
+            // scaling it afterwards gives the maximum of the scaled scores exactly (rounding is
+            // monotone), for a positive scale; a negative scale takes the minimum instead
+            const float c2 = j.scale_log2;
+            const bool pos = c2 >= 0.0f;
+            float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+            for (int c = 0; c < 4; c += 2) {
+                uint32_t v0[32], v1[32];
+                tc_ld32_nowait(scol + 32 * c, v0);
+                tc_ld32_nowait(scol + 32 * c + 32, v1);
+                tc_wait_ld();
+                if (full && pos) {
 #pragma unroll
-        for (int n = 0; n < kBK / 8; ++n) {
-            const float p00 = exp2f(s[n][0] - b0), p01 = exp2f(s[n][1] - b0);
-            const float p10 = exp2f(s[n][2] - b1), p11 = exp2f(s[n][3] - b1);
-            l0 += p00 + p01;
-            l1 += p10 + p11;
-            pa[n >> 1][(n & 1) * 2] = bf16x2(p00, p01);
-            pa[n >> 1][(n & 1) * 2 + 1] = bf16x2(p10, p11);
+                    for (int e = 0; e < 32; ++e) {
+                        xm[e & 3] = fmaxf(xm[e & 3], __uint_as_float(v0[e]));
+                        xm[e & 3] = fmaxf(xm[e & 3], __uint_as_float(v1[e]));
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        if (t0 + 32 * c + e < j.total_tokens)
+                            xm[e & 3] = fmaxf(xm[e & 3], pos ? __uint_as_float(v0[e]) : -__uint_as_float(v0[e]));
+                        if (t0 + 32 * c + 32 + e < j.total_tokens)
+                            xm[e & 3] = fmaxf(xm[e & 3], pos ? __uint_as_float(v1[e]) : -__uint_as_float(v1[e]));
+                    }
+                }
+            }
+            const float xr = fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3]));
+            const float x = xr == -INFINITY ? -INFINITY : (pos ? xr * c2 : -xr * c2);
+            const float mn = fmaxf(m, x);
+            const float b = mn == -INFINITY ? 0.0f : mn;
+            const float alpha = ex2(m - b);
+            // O_t is stable here (s_full(i) implies P.V(i - 1) done): rescale it when any row of
+            // the warp moved its maximum (tcgen05.ld/st are warp-wide)
+            if (i > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t v[32];
+                    tc_ld32_nowait(ocol + 32 * c, v);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+                    tc_st32(ocol + 32 * c, v);
+                }
+            }
+            // pass 2: P = 2^(s * c2 - b) (BF16 pairs) and its row sum, paired FP32 arithmetic; in
+            // two halves of 64 tokens, each written over S columns already read (P half h to
+            // columns [32h, 32h + 32), from S columns [64h, 64h + 64))
+            float2 sum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+#pragma unroll 1
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t p[32];
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * hh + cc;
+                    uint32_t v[32];
+                    tc_ld32_nowait(scol + 32 * c, v);
+                    tc_wait_ld();
+                    if (full) {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 t = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), c2, -b);
+                            const float2 pp = make_float2(ex2(t.x), ex2(t.y));
+                            sum2[(e >> 1) & 1] = add2(sum2[(e >> 1) & 1], pp);
+                            p[16 * cc + e / 2] = bf16x2(pp.x, pp.y);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 t = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), c2, -b);
+                            const float p0 = t0 + 32 * c + e < j.total_tokens ? ex2(t.x) : 0.0f;
+                            const float p1 = t0 + 32 * c + e + 1 < j.total_tokens ? ex2(t.y) : 0.0f;
+                            sum2[(e >> 1) & 1] = add2(sum2[(e >> 1) & 1], make_float2(p0, p1));
+                            p[16 * cc + e / 2] = bf16x2(p0, p1);
+                        }
+                    }
+                }
+                tc_st32(scol + 32 * hh, p);
+            }
+            const float sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
+            l = l * alpha + sum;
+            m = mn;
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(p_full);
         }
-
-        // O += P V
+        if (ok && ntiles > 0 && warp_wait(bar_o_done + 8 * qt, 0)) {
+            tc_fence_after();
+            const float inv = 1.0f / l;
+            const int64_t row = q0 + qt * kBQ + r;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t v[32];
+                tc_ld32_nowait(ocol + 32 * c, v);
+                tc_wait_ld();
+                if (row < j.tq && NVFP4_CHECKED(row * j.ldo + head * kD + 32 * c, 32, j.o_elems, status)) {
+                    uint16_t *dst = j.o + row * j.ldo + head * kD + 32 * c;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-#pragma unroll
-            for (int dp = 0; dp < kD / 16; ++dp) {
-                uint32_t b[4];
-                ldmatrix_x4_trans(vb + (kk * 16 + (mi & 1) * 8 + mr) * kPitch + (dp * 16 + (mi >> 1) * 8) * 2, b);
-                mma_bf16(o[2 * dp], pa[kk], b[0], b[1]);
-                mma_bf16(o[2 * dp + 1], pa[kk], b[2], b[3]);
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 w = make_uint4(
+                            bf16x2(__uint_as_float(v[8 * q + 0]) * inv, __uint_as_float(v[8 * q + 1]) * inv),
+                            bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv),
+                            bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv),
+                            bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv));
+                        *reinterpret_cast<uint4 *>(dst + 8 * q) = w;
+                    }
+                }
             }
         }
     }
 
-    // normalise and store (each row's sum >= 1: its maximum contributes exp2(0))
-    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 1);
-    l0 += __shfl_xor_sync(0xFFFFFFFFu, l0, 2);
-    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 1);
-    l1 += __shfl_xor_sync(0xFFFFFFFFu, l1, 2);
-    const float i0 = 1.0f / l0, i1 = 1.0f / l1;
-#pragma unroll
-    for (int n = 0; n < kD / 8; ++n) {
-        const int c = head * kD + n * 8 + tq4 * 2;
-        if (r0 < j.tq) *reinterpret_cast<uint32_t *>(j.o + r0 * j.ldo + c) = bf16x2(o[n][0] * i0, o[n][1] * i0);
-        if (r1 < j.tq) *reinterpret_cast<uint32_t *>(j.o + r1 * j.ldo + c) = bf16x2(o[n][2] * i1, o[n][3] * i1);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 12) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMEM_COLS) : "memory");
     }
 }
 
 }  // namespace
 
 cudaError_t launch_kv_attention(const AttnJob &j, int32_t *status, cudaStream_t s) {
-    (void)status;                                         // this kernel never waits
     if (j.tq <= 0) return cudaSuccess;
-    static std::atomic<bool> attr_set[64];               // per device; a repeated set is harmless
+    static std::atomic<bool> attr_set[64];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -272,8 +550,8 @@ cudaError_t launch_kv_attention(const AttnJob &j, int32_t *status, cudaStream_t 
         if (e != cudaSuccess) return e;
         attr_set[dev].store(true, std::memory_order_release);
     }
-    const dim3 grid((unsigned)ceil_div(j.tq, kBQ), (unsigned)j.heads);
-    return launch_pdl(kv_attention_kernel, grid, dim3(kThreads), kSmemBytes, s, j);
+    const dim3 grid((unsigned)ceil_div(j.tq, kQTiles * kBQ), (unsigned)j.heads);
+    return launch_pdl(kv_attention_kernel, grid, dim3(kThreads), kSmemBytes, s, j, status);
 }
 
 }  // namespace nvfp4

@@ -12,6 +12,7 @@ struct AttnSlot {
     const uint8_t *sf_k, *sf_v;         // [ntok][row_sf]
     const float *g_k, *g_v;
     int64_t tok_begin;
+    int64_t ntok;                       // tokens the slot holds (extent of its arrays, checked build)
 };
 
 struct AttnJob {
@@ -25,6 +26,7 @@ struct AttnJob {
     uint16_t *o;                        // [tq][ldo] BF16, same column layout
     int64_t ldo;
     float scale_log2;                   // softmax scale * log2(e)
+    int64_t q_elems, o_elems;           // extents of q and o from their starts (checked build)
 };
 
 // head_dim is 128 (checked by the caller).  status: the optional device status word (a bounded

@@ -109,6 +109,9 @@ nvfp4_status gemm_args(const nvfp4_tensor *A, const nvfp4_tensor *B, const void 
     a.ldy = ldy;
     a.y_f32 = y_dtype == NVFP4_OUT_F32;
     a.status = dev_status;
+    a.y_elems = (A->rows - 1) * ldy + B->rows;
+    a.bias_elems = B->rows;
+    a.resid_elems = (A->rows - 1) * ldy + B->rows;
     return NVFP4_OK;
 }
 
@@ -135,6 +138,14 @@ extern "C" {
 
 int32_t nvfp4_version(void) { return 100; }
 
+int32_t nvfp4_checked_build(void) {
+#ifdef NVFP4_DEBUG_CHECKS
+    return 1;
+#else
+    return 0;
+#endif
+}
+
 const char *nvfp4_last_error(void) { return g_last_error; }
 
 const char *nvfp4_status_string(int32_t status) {
@@ -145,6 +156,7 @@ const char *nvfp4_status_string(int32_t status) {
         case NVFP4_ERR_NONFINITE: return "non-finite input";
         case NVFP4_ERR_TIMEOUT: return "bounded on-chip wait timed out";
         case NVFP4_ERR_CUDA: return "CUDA error";
+        case NVFP4_ERR_OUT_OF_BOUNDS: return "checked build: an access outside its buffer was skipped";
         default: return "unknown status";
     }
 }
@@ -198,6 +210,8 @@ nvfp4_status nvfp4_amax(const void *x_bf16, int64_t M, int64_t K, int64_t ld, fl
     jobs.job[0].cols = K;
     jobs.job[0].ld = ld;
     jobs.job[0].partial = static_cast<uint32_t *>(ws);
+    jobs.job[0].status = dev_status;
+    jobs.job[0].x_elems = M > 0 ? (M - 1) * ld + K : 0;
     cudaError_t e = launch_amax(jobs, dev_status, amax_out, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_amax");
 }
@@ -233,6 +247,8 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
     j.ld = ld;
     j.partial = reinterpret_cast<uint32_t *>(scratch);
     j.rec = rec;
+    j.status = dev_status;
+    j.x_elems = (M - 1) * ld + K;
     RecJobs rj{};
     rj.njobs = 1;
     rj.npartial = jobs.npartial;
@@ -246,7 +262,7 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
         // one launch per layout: the quantize passes build the scale record from amax_in
         // themselves; the first pass reports g (both outputs) and a non-finite amax
         j.amax_in = amax_in;
-        j.status = dev_status;
+        j.report_record = 1;
         j.g_out[0] = row_out ? row_out->g : col_out->g;
         j.g_out[1] = row_out && col_out ? col_out->g : nullptr;
     } else {
@@ -258,18 +274,19 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
         j.pitch = codes_pitch(K);
         j.sf = row_out->sf;
         j.sf_layout = row_out->sf_layout;
+        j.codes_bytes = M * codes_pitch(K);
+        j.sf_bytes = sf_bytes(M, K, row_out->sf_layout);
         e = launch_quantize_rows(jobs, s);
     }
     if (e == cudaSuccess && col_out) {
         RowJob jc = j;
-        if (row_out) {                                    // the row pass reported already
-            jc.g_out[0] = jc.g_out[1] = nullptr;
-            jc.status = nullptr;
-        }
+        if (row_out) jc.report_record = 0;                // the row pass reported already
         jc.codes = col_out->codes;
         jc.pitch = codes_pitch(M);
         jc.sf = col_out->sf;
         jc.sf_layout = col_out->sf_layout;
+        jc.codes_bytes = K * codes_pitch(M);
+        jc.sf_bytes = sf_bytes(K, M, col_out->sf_layout);
         e = launch_quantize_cols(jc, row_out != nullptr, s);
     }
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_quantize");
@@ -315,6 +332,8 @@ nvfp4_status nvfp4_gemm_quant_out(const nvfp4_tensor *A, const nvfp4_tensor *B, 
     a.q_sf = q_out->sf;
     a.q_pitch = codes_pitch(B->rows);
     a.q_sf_layout = q_out->sf_layout;
+    a.q_codes_bytes = A->rows * a.q_pitch;
+    a.q_sf_bytes = sf_bytes(A->rows, B->rows, q_out->sf_layout);
     cudaError_t e = launch_scale_record(rj, dev_status, s);
     if (e == cudaSuccess) e = launch_gemm(a, s);
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_gemm_quant_out");
@@ -341,6 +360,7 @@ nvfp4_status nvfp4_gemm_colamax(const nvfp4_tensor *A, const nvfp4_tensor *B, co
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     a.cam_partial = static_cast<uint32_t *>(ws);
     a.cam_n128 = N / 128;
+    a.cam_elems = ceil_div(M, 32) * (N / 128);
     cudaError_t e = launch_gemm(a, s);
     if (e == cudaSuccess)
         e = launch_colamax_finish(a.cam_partial, ceil_div(M, 32), N / 128, group_cols, N / group_cols, amax_out,
@@ -409,6 +429,10 @@ nvfp4_status kv_quant_append_amax(nvfp4_kv_cache *cache, int32_t layer, int32_t 
         j.sf_layout = NVFP4_SF_LINEAR;
         j.partial = reinterpret_cast<uint32_t *>(scratch);
         j.rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
+        j.status = dev_status;
+        j.x_elems = (ntok - 1) * ld + row;
+        j.codes_bytes = ntok * (row / 2);
+        j.sf_bytes = ntok * (row / 16);
         rj.job[i].partial = j.partial;
         rj.job[i].amax_in = amax_kv ? amax_kv + i : nullptr;
         rj.job[i].rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
@@ -417,7 +441,7 @@ nvfp4_status kv_quant_append_amax(nvfp4_kv_cache *cache, int32_t layer, int32_t 
         if (amax_kv) {                                    // one launch: the row pass builds the record
             j.amax_in = amax_kv + i;
             j.g_out[0] = rj.job[i].g_out[0];
-            j.status = dev_status;
+            j.report_record = 1;
         }
     }
     cudaError_t e = cudaSuccess;
@@ -454,9 +478,9 @@ nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, const int32_
         if (len == 0) continue;
         const int64_t tok0 = slot_index * cache->slot_tokens;
         jk.slot[n] = DequantSlot{cache->codes_k + tok0 * (row / 2), cache->sf_k + tok0 * (row / 16),
-                                 cache->g_k + slot_index, tok};
+                                 cache->g_k + slot_index, tok, len};
         jv.slot[n] = DequantSlot{cache->codes_v + tok0 * (row / 2), cache->sf_v + tok0 * (row / 16),
-                                 cache->g_v + slot_index, tok};
+                                 cache->g_v + slot_index, tok, len};
         tok += len;
         ++n;
     }
@@ -466,6 +490,7 @@ nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, const int32_
     jk.row_elems = jv.row_elems = row;
     jk.out = static_cast<uint16_t *>(k_out_bf16);
     jv.out = static_cast<uint16_t *>(v_out_bf16);
+    jk.status = jv.status = dev_status;
     cudaError_t e = launch_kv_dequant(&jk, &jv, dev_status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "kv_dequant");
 }
@@ -496,7 +521,7 @@ nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, const int3
         const int64_t tok0 = slot_index * cache->slot_tokens;
         j.slot[n] = AttnSlot{cache->codes_k + tok0 * (row / 2), cache->codes_v + tok0 * (row / 2),
                              cache->sf_k + tok0 * (row / 16), cache->sf_v + tok0 * (row / 16),
-                             cache->g_k + slot_index, cache->g_v + slot_index, tok};
+                             cache->g_k + slot_index, cache->g_v + slot_index, tok, len};
         tok += len;
         ++n;
     }
@@ -515,6 +540,8 @@ nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, const int3
     j.o = static_cast<uint16_t *>(o_bf16);
     j.ldo = ldo;
     j.scale_log2 = (float)((double)scale * 1.4426950408889634);   // log2(e)
+    j.q_elems = (tq - 1) * ldq + row;
+    j.o_elems = (tq - 1) * ldo + row;
     cudaError_t e = launch_kv_attention(j, dev_status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "kv_attention");
 }
@@ -534,6 +561,15 @@ nvfp4_status nvfp4_selftest_wait_timeout(int32_t *dev_status, int64_t limit_ns, 
     if (st != NVFP4_OK) return st;
     cudaError_t e = launch_wait_timeout(dev_status, limit_ns, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_selftest_wait_timeout");
+}
+
+nvfp4_status nvfp4_selftest_bounds(uint8_t *buf, int64_t extent, int64_t index, int32_t *dev_status,
+                                   nvfp4_stream stream) {
+    if (!buf || extent < 0 || index < 0) return NVFP4_ERR_INVALID_ARG;
+    nvfp4_status st = check_device();
+    if (st != NVFP4_OK) return st;
+    cudaError_t e = launch_bounds_selftest(buf, extent, index, dev_status, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "nvfp4_selftest_bounds");
 }
 
 }  // extern "C"

@@ -42,6 +42,26 @@ __device__ __forceinline__ void set_status(int32_t *st, int32_t code) {
     if (st) atomicCAS(st, 0, code);
 }
 
+// ---- checked build ------------------------------------------------------------------------------
+//
+// Compiled with NVFP4_DEBUG_CHECKS, NVFP4_CHECKED(off, len, extent, status) is true when the access
+// [off, off + len) lies inside a buffer of `extent` units (elements or bytes, as the call site
+// states) and otherwise writes NVFP4_ERR_OUT_OF_BOUNDS to the status word and returns false, so
+// the caller skips the access.  The extents come from the host, computed from the tensor shapes
+// the caller declared, independently of the kernels' index arithmetic.  In the release build the
+// macro is the constant true and compiles away.
+#ifdef NVFP4_DEBUG_CHECKS
+__device__ __forceinline__ bool dbg_in_bounds(int64_t off, int64_t len, int64_t extent, int32_t *status) {
+    if (off >= 0 && len >= 0 && off <= extent - len) return true;
+    set_status(status, NVFP4_ERR_OUT_OF_BOUNDS);
+    return false;
+}
+#define NVFP4_CHECKED(off, len, extent, status) \
+    ::nvfp4::dbg_in_bounds((int64_t)(off), (int64_t)(len), (int64_t)(extent), (status))
+#else
+#define NVFP4_CHECKED(off, len, extent, status) true
+#endif
+
 // ---- conversions ------------------------------------------------------------------------------
 
 // Eight FP32 -> 32 bits of packed E2M1 codes, element 0 in the lowest nibble.

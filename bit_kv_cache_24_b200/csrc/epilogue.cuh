@@ -26,8 +26,8 @@ __device__ __forceinline__ void load_record_plain(const ScaleRecord *rec, SmemRe
 // The two scale bytes of 16-blocks blk and blk + 1 (blk even) of row m, adjacent in both layouts.
 __device__ __forceinline__ void store_sf_pair(const GemmArgs &a, int64_t m, int64_t blk, uint32_t two) {
     const int64_t nb = a.N >> 4;
-    uint8_t *p = a.q_sf_layout ? a.q_sf + sf_mma_offset(m, blk, (nb + 3) >> 2) : a.q_sf + m * nb + blk;
-    *reinterpret_cast<uint16_t *>(p) = (uint16_t)two;
+    const int64_t off = a.q_sf_layout ? sf_mma_offset(m, blk, (nb + 3) >> 2) : m * nb + blk;
+    if (NVFP4_CHECKED(off, 2, a.q_sf_bytes, a.status)) *reinterpret_cast<uint16_t *>(a.q_sf + off) = (uint16_t)two;
 }
 
 // Row-wise NVFP4 of one 32-column chunk of output row m (columns n0 .. n0 + 31, n0 % 32 == 0,
@@ -38,7 +38,8 @@ __device__ __forceinline__ void emit_nvfp4_chunk(const GemmArgs &a, const SmemRe
     uint32_t c0, c1, s0, c2, c3, s1;
     quantize16(w, rec, c0, c1, s0);
     quantize16(w + 8, rec, c2, c3, s1);
-    *reinterpret_cast<uint4 *>(a.q_codes + m * a.q_pitch + (n0 >> 1)) = make_uint4(c0, c1, c2, c3);
+    if (NVFP4_CHECKED(m * a.q_pitch + (n0 >> 1), 16, a.q_codes_bytes, a.status))
+        *reinterpret_cast<uint4 *>(a.q_codes + m * a.q_pitch + (n0 >> 1)) = make_uint4(c0, c1, c2, c3);
     store_sf_pair(a, m, n0 >> 4, s0 | (s1 << 8));
 }
 

@@ -328,7 +328,7 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 if (args.bias) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        if (n0 + 8 * q >= N) break;
+                        if (n0 + 8 * q >= N || !NVFP4_CHECKED(n0 + 8 * q, 8, args.bias_elems, args.status)) break;
                         const uint4 b = ldg_v4(args.bias + n0 + 8 * q);
                         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -340,7 +340,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 } else if (args.resid) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        if (n0 + 8 * q >= N) break;
+                        if (n0 + 8 * q >= N ||
+                            !NVFP4_CHECKED(m * args.ldy + n0 + 8 * q, 8, args.resid_elems, args.status))
+                            break;
                         const uint4 b = ldg_v4(args.resid + m * args.ldy + n0 + 8 * q);
                         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -358,7 +360,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                         uint16_t *yrow = reinterpret_cast<uint16_t *>(args.y) + m * args.ldy + n0;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            if (n0 + 8 * q >= N) break;
+                            if (n0 + 8 * q >= N || !NVFP4_CHECKED(m * args.ldy + n0 + 8 * q, 8, args.y_elems, args.status))
+                                break;
                             stg_v4(yrow + 8 * q, make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]));
                         }
                     }
@@ -372,7 +375,8 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                     float *yrow = reinterpret_cast<float *>(args.y) + m * args.ldy + n0;
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
-                        if (n0 + 4 * q >= N) break;
+                        if (n0 + 4 * q >= N || !NVFP4_CHECKED(m * args.ldy + n0 + 4 * q, 4, args.y_elems, args.status))
+                            break;
                         stg_v4(yrow + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
                                                         __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
                     }
@@ -387,8 +391,12 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
                 const int64_t r32 = ((int64_t)mb * BM + sub * 32) >> 5;
                 const int64_t c128 = ((int64_t)nb * BN) >> 7;
                 if (lane == 0 && r32 < ceil_div(M, 32)) {
-                    if (c128 < args.cam_n128) args.cam_partial[r32 * args.cam_n128 + c128] = cam0;
-                    if (c128 + 1 < args.cam_n128) args.cam_partial[r32 * args.cam_n128 + c128 + 1] = cam1;
+                    if (c128 < args.cam_n128 &&
+                        NVFP4_CHECKED(r32 * args.cam_n128 + c128, 1, args.cam_elems, args.status))
+                        args.cam_partial[r32 * args.cam_n128 + c128] = cam0;
+                    if (c128 + 1 < args.cam_n128 &&
+                        NVFP4_CHECKED(r32 * args.cam_n128 + c128 + 1, 1, args.cam_elems, args.status))
+                        args.cam_partial[r32 * args.cam_n128 + c128 + 1] = cam1;
                 }
             }
             tc_fence_before();

@@ -391,10 +391,15 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
                     for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(alpha, __uint_as_float(r[c][i]));
                     const uint16_t *addsrc = args.bias ? args.bias + n0
                                                        : (args.resid && row_ok ? args.resid + m * args.ldy + n0 : nullptr);
+                    const int64_t addoff = args.bias ? n0 : m * args.ldy + n0;      // checked build
+                    const int64_t addext = args.bias ? args.bias_elems : args.resid_elems;
+                    (void)addoff;
+                    (void)addext;
                     if (addsrc) {
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
                             if (n0 + 8 * g >= N) break;
+                            if (!NVFP4_CHECKED(addoff + 8 * g, 8, addext, args.status)) break;
                             const uint4 b = ldg_v4(addsrc + 8 * g);
                             const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -441,10 +446,15 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(alpha, __uint_as_float(r[c][i]));
                 const uint16_t *addsrc = args.bias ? args.bias + n0 : (args.resid ? args.resid + m * args.ldy + n0 : nullptr);
+                const int64_t addoff = args.bias ? n0 : m * args.ldy + n0;          // checked build
+                const int64_t addext = args.bias ? args.bias_elems : args.resid_elems;
+                (void)addoff;
+                (void)addext;
                 if (addsrc) {
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         if (n0 + 8 * g >= N) break;
+                        if (!NVFP4_CHECKED(addoff + 8 * g, 8, addext, args.status)) break;
                         const uint4 b = ldg_v4(addsrc + 8 * g);
                         const uint32_t bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
@@ -462,7 +472,8 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
                         uint16_t *yrow = reinterpret_cast<uint16_t *>(args.y) + m * args.ldy + n0;
 #pragma unroll
                         for (int g = 0; g < 4; ++g) {
-                            if (n0 + 8 * g >= N) break;
+                            if (n0 + 8 * g >= N || !NVFP4_CHECKED(m * args.ldy + n0 + 8 * g, 8, args.y_elems, args.status))
+                                break;
                             stg_v4(yrow + 8 * g, make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]));
                         }
                     }
@@ -472,7 +483,8 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
                     float *yrow = reinterpret_cast<float *>(args.y) + m * args.ldy + n0;
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
-                        if (n0 + 4 * g >= N) break;
+                        if (n0 + 4 * g >= N || !NVFP4_CHECKED(m * args.ldy + n0 + 4 * g, 4, args.y_elems, args.status))
+                            break;
                         stg_v4(yrow + 4 * g, make_uint4(__float_as_uint(v[4 * g]), __float_as_uint(v[4 * g + 1]),
                                                         __float_as_uint(v[4 * g + 2]), __float_as_uint(v[4 * g + 3])));
                     }
@@ -484,7 +496,8 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
                 const int64_t r32 = ((int64_t)mb * BM + (int64_t)rank * BM_CTA + q * 32) >> 5;
                 const int64_t c128 = ((int64_t)nb * BN + half * 128) >> 7;
                 if (lane == 0 && r32 < ceil_div(M, 32) && c128 < args.cam_n128)
-                    args.cam_partial[r32 * args.cam_n128 + c128] = cam;
+                    if (NVFP4_CHECKED(r32 * args.cam_n128 + c128, 1, args.cam_elems, args.status))
+                        args.cam_partial[r32 * args.cam_n128 + c128] = cam;
             }
             acc_phase ^= 1;
         }

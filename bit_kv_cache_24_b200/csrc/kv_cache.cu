@@ -115,7 +115,8 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const __grid_const
                 const int64_t t = r[u] - sl.tok_begin;
                 const int64_t el = e[u] + lane * 32;
                 gv[u] = *sl.g;
-                if (el < j.row_elems) {
+                if (el < j.row_elems && NVFP4_CHECKED(t * row_bytes + (el >> 1), 16, sl.ntok * row_bytes, j.status) &&
+                    NVFP4_CHECKED(t * row_sf + (el >> 4), 2, sl.ntok * row_sf, j.status)) {
                     cw[u] = ldg_nc_v4(sl.codes + t * row_bytes + (el >> 1));
                     sfw[u] = ldg_nc_u16(sl.sf + t * row_sf + (el >> 4));
                 }
@@ -138,7 +139,8 @@ __global__ void __launch_bounds__(kThreads) kv_dequant_kernel(const __grid_const
         for (int u = 0; u < kItems; ++u) {
             if (it0 + u >= items) break;
             const int64_t n = j.row_elems - e[u] < kSpan ? j.row_elems - e[u] : kSpan;
-            bulk_store(j.out + r[u] * j.row_elems + e[u], smem_addr(&stage[warp][u][0]), (uint32_t)(n * 2));
+            if (NVFP4_CHECKED(r[u] * j.row_elems + e[u], n, j.total_tokens * j.row_elems, j.status))
+                bulk_store(j.out + r[u] * j.row_elems + e[u], smem_addr(&stage[warp][u][0]), (uint32_t)(n * 2));
         }
     }
     bulk_wait_all();                                      // stores done before shared memory goes away

@@ -35,11 +35,15 @@ struct RowJob {
     uint32_t *partial;      // [kMaxPartials] partial maxima (BF16 magnitude bits), amax pass
     const ScaleRecord *rec; // read by the quantize passes (unless amax_in is set)
     // Given amax (device float, nullable): the quantize pass builds its scale record itself
-    // (no record kernel) and its first CTA writes g to g_out[] (nullable) or, for a non-finite
-    // amax, NVFP4_ERR_NONFINITE to status.
+    // (no record kernel) and, when report_record is set, its first CTA writes g to g_out[]
+    // (nullable) or, for a non-finite amax, NVFP4_ERR_NONFINITE to status.
     const float *amax_in;
     float *g_out[2];
+    int32_t report_record;
     int32_t *status;
+    // buffer extents for the checked build (see NVFP4_CHECKED): elements of x from its start,
+    // bytes of codes and of sf
+    int64_t x_elems, codes_bytes, sf_bytes;
 };
 
 struct RowJobs {
@@ -91,6 +95,7 @@ struct DequantSlot {
     const uint8_t *sf;      // [ntok][row_sf]
     const float *g;
     int64_t tok_begin;      // first output token of this slot
+    int64_t ntok;           // tokens the slot holds (extent of codes and sf, checked build)
 };
 
 constexpr int kMaxDequantSlots = 128;
@@ -101,6 +106,7 @@ struct DequantJob {
     int64_t total_tokens;
     int64_t row_elems;      // heads * head_dim
     uint16_t *out;          // [total_tokens][row_elems]
+    int32_t *status;        // status word (checked build)
 };
 
 cudaError_t launch_kv_dequant(const DequantJob *k, const DequantJob *v, int32_t *status, cudaStream_t s);
@@ -127,6 +133,9 @@ struct GemmArgs {
     // 128-column block, at cam_partial[(row / 32) * cam_n128 + col / 128] (N % 256 == 0)
     uint32_t *cam_partial;
     int64_t cam_n128;
+    // buffer extents for the checked build (elements of y, bias and resid; bytes of q_codes and
+    // q_sf; words of cam_partial)
+    int64_t y_elems, bias_elems, resid_elems, q_codes_bytes, q_sf_bytes, cam_elems;
 };
 
 // Column-group amax from the GEMM's block partials: amax_out[g] = max over the blocks of columns
@@ -140,6 +149,7 @@ cudaError_t launch_gemm_2sm(const GemmArgs &args, cudaStream_t s);
 
 cudaError_t launch_encode_elements(const float *in, int64_t n, uint8_t *e2m1_out, uint8_t *e4m3_out, cudaStream_t s);
 cudaError_t launch_wait_timeout(int32_t *status, int64_t limit_ns, cudaStream_t s);
+cudaError_t launch_bounds_selftest(uint8_t *buf, int64_t extent, int64_t index, int32_t *status, cudaStream_t s);
 
 int num_sms();
 

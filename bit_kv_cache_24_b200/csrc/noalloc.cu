@@ -121,6 +121,11 @@ nvfp4_status nvfp4_quantize_noalloc(const void *x_bf16, int64_t M, int64_t K, in
     j.sf_layout = out->sf_layout;
     j.partial = reinterpret_cast<uint32_t *>(scratch);
     j.rec = reinterpret_cast<ScaleRecord *>(scratch + kRecordOffset);
+    j.status = dev_status;
+    j.x_elems = (M - 1) * ld + K;
+    j.codes_bytes = orows * j.pitch;
+    j.sf_bytes = out->sf_layout == NVFP4_SF_MMA ? 128 * ceil_div(orows, 128) * 4 * ceil_div(ceil_div(ocols, 16), 4)
+                                                : orows * ceil_div(ocols, 16);
     RecJobs rj{};
     rj.njobs = 1;
     rj.npartial = npartial;

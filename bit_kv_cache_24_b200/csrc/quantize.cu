@@ -144,7 +144,12 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const __grid_con
             if (u < total) {
                 const uint32_t row = flat ? 0u : u / upr;
                 const int64_t off = flat ? (int64_t)u * kElems : (int64_t)row * j.ld + (int64_t)(u - row * upr) * kElems;
-                v[k] = ldg_unit<kWords>(j.x + off);
+                if (NVFP4_CHECKED(off, kElems, j.x_elems, j.status)) {
+                    v[k] = ldg_unit<kWords>(j.x + off);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < kWords; ++i) v[k].w[i] = 0;
+                }
             } else {
 #pragma unroll
                 for (int i = 0; i < kWords; ++i) v[k].w[i] = 0;
@@ -164,7 +169,7 @@ __global__ void __launch_bounds__(kThreads) amax_partial_kernel(const __grid_con
     if (threadIdx.x == 0) {
         uint32_t r = 0;
         for (int w = 0; w < kWarps; ++w) r = max(r, red[w]);
-        j.partial[blockIdx.x] = r;
+        if (NVFP4_CHECKED(blockIdx.x, 1, kMaxPartials, j.status)) j.partial[blockIdx.x] = r;
     }
 }
 
@@ -205,7 +210,8 @@ __global__ void __launch_bounds__(kThreads) colamax_finish_kernel(const uint32_t
 #pragma unroll
             for (int u = 0; u < kRowsInFlight; ++u) {
                 const int64_t r = r0 + (int64_t)u * kWarps;
-                v[u] = r < rows32 ? p[r * n128 + c] : 0u;
+                v[u] = r < rows32 && NVFP4_CHECKED((int64_t)blockIdx.x * cpg + r * n128 + c, 1, rows32 * n128, status)
+                           ? p[r * n128 + c] : 0u;
             }
 #pragma unroll
             for (int u = 0; u < kRowsInFlight; ++u) m = max(m, v[u]);
@@ -289,7 +295,8 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_co
     const uint16_t *xr = j.x + (int64_t)row * j.ld + 64 * q;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-        if (live && 4 * q + b < nb) {
+        if (live && 4 * q + b < nb &&
+            NVFP4_CHECKED((int64_t)row * j.ld + 64 * q + 16 * b, 16, j.x_elems, j.status)) {
             if constexpr (kV8) {
                 const Unit<8> u = ldg_unit<8>(xr + 16 * b);
 #pragma unroll
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_co
         }
     }
     if (j.amax_in)
-        build_record(*j.amax_in, rec, blockIdx.x == 0, j.g_out[0], j.g_out[1], j.status);
+        build_record(*j.amax_in, rec, j.report_record && blockIdx.x == 0, j.g_out[0], j.g_out[1], j.status);
     else
         load_record(j.rec, rec);
     __syncthreads();
@@ -319,20 +326,24 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_co
         sfw |= sf << (8 * b);
     }
     if (live) {
-        uint8_t *cr = j.codes + (int64_t)row * j.pitch + 32 * q;
-        if (32 * q < j.pitch) stg_v4(cr, c[0], c[1], c[2], c[3]);
-        if (32 * q + 16 < j.pitch) stg_v4(cr + 16, c[4], c[5], c[6], c[7]);
+        const int64_t co = (int64_t)row * j.pitch + 32 * q;
+        uint8_t *cr = j.codes + co;
+        if (32 * q < j.pitch && NVFP4_CHECKED(co, 16, j.codes_bytes, j.status)) stg_v4(cr, c[0], c[1], c[2], c[3]);
+        if (32 * q + 16 < j.pitch && NVFP4_CHECKED(co + 16, 16, j.codes_bytes, j.status))
+            stg_v4(cr + 16, c[4], c[5], c[6], c[7]);
     }
     if constexpr (kMma) {
-        *reinterpret_cast<uint32_t *>(j.sf + sf_mma_offset(row, 4 * q, nq)) = sfw;
+        const int64_t so = sf_mma_offset(row, 4 * q, nq);
+        if (NVFP4_CHECKED(so, 4, j.sf_bytes, j.status)) *reinterpret_cast<uint32_t *>(j.sf + so) = sfw;
     } else if (live) {
-        uint8_t *sr = j.sf + (int64_t)row * nb + 4 * q;
+        const int64_t so = (int64_t)row * nb + 4 * q;
+        uint8_t *sr = j.sf + so;
         if (4 * q + 3 < nb && ((reinterpret_cast<uintptr_t>(sr) & 3) == 0)) {
-            *reinterpret_cast<uint32_t *>(sr) = sfw;
+            if (NVFP4_CHECKED(so, 4, j.sf_bytes, j.status)) *reinterpret_cast<uint32_t *>(sr) = sfw;
         } else {
 #pragma unroll
             for (int b = 0; b < 4; ++b)
-                if (4 * q + b < nb) sr[b] = (uint8_t)(sfw >> (8 * b));
+                if (4 * q + b < nb && NVFP4_CHECKED(so + b, 1, j.sf_bytes, j.status)) sr[b] = (uint8_t)(sfw >> (8 * b));
         }
     }
 }
@@ -376,15 +387,15 @@ __device__ __forceinline__ void cols_body(const RowJob &j, SmemRecord &rec) {
     for (int r = 0; r < 16; ++r) {
         const uint32_t m = m0 + r;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (active && m < M && k0 < K) {
+        if (active && m < M && k0 < K && NVFP4_CHECKED((int64_t)m * j.ld + k0, 8, j.x_elems, j.status)) {
             const uint16_t *p = j.x + (int64_t)m * j.ld + k0;
             v = kConcurrent ? ldg_cg_v4(p) : ldg_nc_v4(p);
         }
         w[r][0] = v.x; w[r][1] = v.y; w[r][2] = v.z; w[r][3] = v.w;
     }
     if (j.amax_in)   // concurrent: complete before the row pass started, read through L2
-        build_record(kConcurrent ? __uint_as_float(ldg_cg_u32(j.amax_in)) : *j.amax_in, rec, blockIdx.x == 0,
-                     j.g_out[0], j.g_out[1], j.status);
+        build_record(kConcurrent ? __uint_as_float(ldg_cg_u32(j.amax_in)) : *j.amax_in, rec,
+                     j.report_record && blockIdx.x == 0, j.g_out[0], j.g_out[1], j.status);
     else
         load_record<kConcurrent>(j.rec, rec);
     __syncthreads();
@@ -401,11 +412,14 @@ __device__ __forceinline__ void cols_body(const RowJob &j, SmemRecord &rec) {
             uint32_t c0, c1, sf;
             quantize16(b, rec, c0, c1, sf);
             if (k < K) {
-                if (m0 < code_cols)
-                    *reinterpret_cast<uint2 *>(j.codes + (int64_t)k * j.pitch + (m0 >> 1)) = make_uint2(c0, c1);
-                if (!mma && mb < nb) j.sf[(int64_t)k * nb + mb] = (uint8_t)sf;
+                const int64_t co = (int64_t)k * j.pitch + (m0 >> 1);
+                if (m0 < code_cols && NVFP4_CHECKED(co, 8, j.codes_bytes, j.status))
+                    *reinterpret_cast<uint2 *>(j.codes + co) = make_uint2(c0, c1);
+                if (!mma && mb < nb && NVFP4_CHECKED((int64_t)k * nb + mb, 1, j.sf_bytes, j.status))
+                    j.sf[(int64_t)k * nb + mb] = (uint8_t)sf;
             }
-            if (mma) j.sf[sf_mma_offset(k, mb, atoms)] = (uint8_t)sf;
+            if (mma && NVFP4_CHECKED(sf_mma_offset(k, mb, atoms), 1, j.sf_bytes, j.status))
+                j.sf[sf_mma_offset(k, mb, atoms)] = (uint8_t)sf;
         }
     }
 }
@@ -444,6 +458,13 @@ __global__ void wait_timeout_kernel(int32_t *status, int64_t limit_ns) {
     if (threadIdx.x == 0) {
         if (!mbar_wait_bounded(a, 0, nullptr, (uint64_t)limit_ns)) set_status(status, NVFP4_ERR_TIMEOUT);
     }
+}
+
+// Test support: one guarded byte write (see nvfp4_selftest_bounds).
+__global__ void bounds_selftest_kernel(uint8_t *buf, int64_t extent, int64_t index, int32_t *status) {
+    (void)extent;
+    (void)status;
+    if (NVFP4_CHECKED(index, 1, extent, status)) buf[index] = 0xAB;
 }
 
 bool all_v8(const RowJobs &jobs) {
@@ -510,6 +531,11 @@ cudaError_t launch_quantize_cols(const RowJob &j, bool after_rows, cudaStream_t 
 cudaError_t launch_encode_elements(const float *in, int64_t n, uint8_t *e2m1_out, uint8_t *e4m3_out, cudaStream_t s) {
     if (n <= 0) return cudaSuccess;
     encode_elements_kernel<<<(unsigned)ceil_div(n, 256), 256, 0, s>>>(in, n, e2m1_out, e4m3_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bounds_selftest(uint8_t *buf, int64_t extent, int64_t index, int32_t *status, cudaStream_t s) {
+    bounds_selftest_kernel<<<1, 1, 0, s>>>(buf, extent, index, status);
     return cudaGetLastError();
 }
 

@@ -60,7 +60,9 @@ typedef enum {
     NVFP4_ERR_UNSUPPORTED = 2,  /* alignment, stride, layout or GPU architecture not supported */
     NVFP4_ERR_NONFINITE = 3,    /* device side: inf/NaN in the input */
     NVFP4_ERR_TIMEOUT = 4,      /* device side: a bounded wait gave up */
-    NVFP4_ERR_CUDA = 5          /* a CUDA runtime/driver call failed */
+    NVFP4_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed */
+    NVFP4_ERR_OUT_OF_BOUNDS = 6 /* device side, checked build only: an access outside its buffer
+                                   was skipped (see nvfp4_checked_build) */
 } nvfp4_status;
 
 typedef enum { NVFP4_ROWWISE = 0, NVFP4_COLWISE = 1, NVFP4_ROWCOL = 2 } nvfp4_dir;
@@ -271,10 +273,13 @@ NVFP4_API nvfp4_status kv_dequant(const nvfp4_kv_cache *cache, int32_t layer, co
  *   scale: the softmax scale (commonly 1 / sqrt(head_dim)), finite.
  * Requires head_dim == 128, ldq and ldo >= heads * head_dim and multiples of 8, q and o 16-byte
  * aligned, a window of at least one token (else NVFP4_ERR_INVALID_ARG / NVFP4_ERR_UNSUPPORTED).
- * tq == 0 is a no-op. dev_status may be NULL: the kernel has no data-dependent error (it never
- * waits), and scores must stay finite in FP32 (|scale * q.k| < 2^127) for a finite result.
- * Arithmetic: FP32 scores and output accumulation, the probabilities rounded to BF16 for the
- * P.V product, the output rounded to BF16 (nearest even).
+ * tq == 0 is a no-op. Scores must stay finite in FP32 (|scale * q.k| < 2^127) for a finite
+ * result.  dev_status (nullable): the kernel's on-chip waits are time-bounded, and one that gives
+ * up writes NVFP4_ERR_TIMEOUT there (the output is then unspecified).
+ * Arithmetic (tcgen05 tensor cores): FP32 scores and output accumulation in tensor memory, the
+ * probabilities 2^(scale * log2(e) * s - max) from the hardware exp2 approximation (results below
+ * 2^-126 flush to 0) rounded to BF16 for the P.V product, the row sums in FP32, the output
+ * rounded to BF16 (nearest even).
  */
 NVFP4_API nvfp4_status kv_attention(const nvfp4_kv_cache *cache, int32_t layer, const int32_t *slots,
                                     int32_t nslots, const void *q_bf16, int64_t tq, int64_t ldq, float scale,
@@ -312,6 +317,16 @@ NVFP4_API const char *nvfp4_last_error(void);
 NVFP4_API int32_t nvfp4_version(void);
 
 /*
+ * 1 for the bounds-checked debug build (libnvfp4_checked.so, compiled with NVFP4_DEBUG_CHECKS),
+ * 0 for the release build.  In the checked build every kernel access whose address is computed
+ * from indexes is compared with the extent of its buffer, derived on the host from the caller's
+ * tensor shapes; an access outside it is skipped and NVFP4_ERR_OUT_OF_BOUNDS is written to the
+ * status word instead (no trap, the CUDA context stays usable).  TMA tensor loads and stores are
+ * bounded by their tensor maps and need no check.  Same ABI and results otherwise; slower.
+ */
+NVFP4_API int32_t nvfp4_checked_build(void);
+
+/*
  * Test support: element-wise hardware encoders of the CUDA path on n FP32 inputs:
  * e2m1_out[i] = E2M1 code of in[i] as the quantizer computes it, e4m3_out[i] = E4M3 byte of
  * |in[i]| as the scale step computes it (either output may be NULL).  Device pointers.
@@ -326,6 +341,16 @@ NVFP4_API nvfp4_status nvfp4_encode_elements(const float *in, int64_t n, uint8_t
  */
 NVFP4_API nvfp4_status nvfp4_selftest_wait_timeout(int32_t *dev_status, int64_t limit_ns,
                                          nvfp4_stream stream);
+
+/*
+ * Test support for the checked build: one device thread writes 0xAB to buf[index] if index lies
+ * inside [0, extent) -- in the checked build that comparison is the library's bounds check, which
+ * skips the write and sets NVFP4_ERR_OUT_OF_BOUNDS in *dev_status otherwise; the release build
+ * writes unconditionally.  The caller's buffer must hold index + 1 bytes either way (the test
+ * declares a smaller extent than it allocates), so no call of it can write outside memory.
+ */
+NVFP4_API nvfp4_status nvfp4_selftest_bounds(uint8_t *buf, int64_t extent, int64_t index, int32_t *dev_status,
+                                             nvfp4_stream stream);
 
 #ifdef __cplusplus
 }

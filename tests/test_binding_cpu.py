@@ -28,3 +28,16 @@ def test_kv_attention_marshalling_errors():
     cache = nv.KVCache(1, 2, 128, 2, 16, "cpu")                               # storage only; never launched
     with pytest.raises(TypeError):
         nv.kv_attention(cache, 0, [0], torch.zeros(4, 2, 128, dtype=torch.bfloat16), 1.0)
+
+
+def test_status_word_marshalling(monkeypatch):
+    """The caller's status word is passed through; the release build adds none of its own; the
+    checked build (here faked, no GPU needed for the release path) is what enables the binding's
+    own words."""
+    assert nv.checked_build() is False                     # the in-tree release build
+    assert nv._status(None) is None
+    t = torch.zeros(1, dtype=torch.int32)
+    assert nv._status(t).value == t.data_ptr()
+    assert nv.checked_status() == 0                        # nothing was ever handed out
+    monkeypatch.setattr(nv, "_checked", True)
+    assert nv._status(t).value == t.data_ptr()             # an explicit word always wins

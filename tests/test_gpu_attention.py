@@ -6,8 +6,9 @@ Tolerance, from the kernel's arithmetic (per head h, output column c):
 - The probabilities are rounded to BF16 for the P.V product while their sum stays FP32. This
   perturbs each weight by at most 2^-9 relative, hence O by at most 2^-9 * max_j |v[j, h, c]|.
 - The output is rounded to BF16, adding at most 2^-9 * |O|.
-- The FP32 accumulation of scores and products and exp2 stay orders of magnitude below these
-  two terms at these sizes.
+- The FP32 accumulation of scores and products and the hardware exp2 approximation (relative
+  error ~2^-22; results below 2^-126 flush to 0) stay orders of magnitude below these two terms
+  at these sizes.
 The K and V the kernel multiplies are the restore's values bit for bit (same rounding steps), so
 a one-token window returns that token's V exactly.
 """
@@ -53,6 +54,7 @@ def _fill(orc, heads, lens, seed=0):
     (1, (64, 64, 64), (0, 1, 2), 64),        # tile-aligned window, one full CTA
     (2, (200, 0, 17), (2, 1, 0), 129),       # an empty slot, 3 CTAs with a one-row tail
     (3, (5,), (0,), 3),                      # window shorter than a tile
+    (2, (130, 260), (0, 1), 300),            # two CTAs of two 128-row Q tiles, the last partly live
 ])
 def test_matches_oracle(orc, heads, lens, order, tq):
     cache, model = _fill(orc, heads, lens)
@@ -130,3 +132,15 @@ def test_argument_errors(orc):
     # no queries: nothing to do
     out = nv.kv_attention(cache, 0, [0], q[:0], 1.0)
     assert out.shape == (0, 2, D)
+
+
+def test_negative_scale(orc):
+    # the row maximum of scale * s is the scale times the row minimum of s when scale < 0
+    heads = 2
+    cache, model = _fill(orc, heads, (100, 40), seed=3)
+    q = synth.normal(11, 0, (50, heads, D))
+    o = nv.kv_attention(cache, 0, [0, 1], q.cuda(), -0.06)
+    torch.cuda.synchronize()
+    ref = model.attention(0, [0, 1], q, -0.06)
+    _, vbits = model.dequant(0, [0, 1])
+    _tol_check(o.float().cpu().numpy(), ref, orc.bf16_bits_to_f32(vbits))
