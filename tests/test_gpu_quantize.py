@@ -117,10 +117,15 @@ def test_full_size_ffn_down_activation(orc):
 
 
 @pytest.mark.parametrize("rows,cols,kind", [(1, 16, "normal"), (37, 48, "outliers"), (300, 96, "wide"),
-                                            (1040, 512, "lognormal"), (4680, 3072, "lognormal"), (6000, 256, "normal")])
+                                            (1040, 512, "lognormal"), (4680, 3072, "lognormal"), (6000, 256, "normal"),
+                                            # cols % 64 == 0: the single-read kernel, ragged rows, row-wise
+                                            # padding rows beyond the column layout's padded range
+                                            (1, 64, "normal"), (17, 128, "outliers"), (129, 64, "wide"),
+                                            (200, 192, "lognormal"), (2049, 320, "outliers")])
 @pytest.mark.parametrize("layout", [nv.SF_LINEAR, nv.SF_MMA])
 def test_rowcol_from_one_read(orc, rows, cols, kind, layout):
-    """NVFP4_ROWCOL: row-wise and column-wise outputs of one call equal the oracle's, byte for byte."""
+    """NVFP4_ROWCOL: row-wise and column-wise outputs of one call equal the oracle's, byte for byte
+    (for cols % 64 == 0 from one kernel that reads x once, otherwise a row pass and a column pass)."""
     x = synth.ragged(rows * 5 + cols, rows, cols, kind)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     gr, gc = nv.nvfp4_quantize(x.cuda(), nv.ROWCOL, sf_layout=layout, status=st)
@@ -185,3 +190,20 @@ def test_nonfinite_amax_in_sets_status_and_writes_nothing(direction):
         assert st.item() == nv.NVFP4_ERR_NONFINITE
         for q in outs:
             assert bool((q.codes == 0xAB).all()) and bool((q.sf == 0xCD).all()) and q.g.item() == -1.0
+
+
+@pytest.mark.parametrize("rows,cols", [(129, 64), (4680, 3072), (33, 192)])
+def test_rowcol_mixed_scale_layouts(orc, rows, cols):
+    """Both layouts from one call with different scale layouts for the two outputs (tensor-core
+    layout row-wise, linear column-wise, and the reverse)."""
+    x = synth.ragged(rows + 7 * cols, rows, cols, "lognormal")
+    _, orow = orc.quantize(x)
+    _, ocol = orc.quantize(x, colwise=True)
+    for lr, lc in ((nv.SF_MMA, nv.SF_LINEAR), (nv.SF_LINEAR, nv.SF_MMA)):
+        out = (nv.QTensor(rows, cols, lr), nv.QTensor(cols, rows, lc))
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        nv.nvfp4_quantize(x.cuda(), nv.ROWCOL, out=out, status=st)
+        torch.cuda.synchronize()
+        assert st.item() == 0
+        assert_quantized_equal(orc, out[0], orow, f"mixed row {lr}")
+        assert_quantized_equal(orc, out[1], ocol, f"mixed col {lc}")
