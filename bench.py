@@ -386,6 +386,30 @@ class QKVStep:
         }
 
 
+def attention_on_step_window(st, bf16_peak, reps=10):
+    """kv_attention of the step's queries (the Q third of its QKV output, row stride 9216) over
+    the step's 12-slot NVFP4 window (56160 tokens x 24 heads x 128), timed outside the step:
+    device time per launch, mean of `reps` launches after 3 warm-up launches."""
+    nv = st.nv
+    q = st.Y[:, :HID]
+    o = torch.empty(M_TOK, HEADS * HEAD_DIM, dtype=torch.bfloat16, device=st.Y.device)
+    slots, scale = list(range(SLOTS)), 1.0 / math.sqrt(HEAD_DIM)
+    for _ in range(3):
+        nv.kv_attention(st.cache, 0, slots, q, scale, out=o, status=st.status)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        nv.kv_attention(st.cache, 0, slots, q, scale, out=o, status=st.status)
+    b.record()
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / 1e3 / reps
+    tf = ATTN_FLOP / t / 1e12
+    return {"bound": "tensor", "us_per_launch": round(t * 1e6, 1), "achieved": round(tf, 1), "unit": "TFLOP/s",
+            "peak": round(bf16_peak, 1), "frac": round(tf / bf16_peak, 4), "share": None,
+            "stream": "outside the step: the step's Q over its 12-slot NVFP4 window (restore fused), mean of "
+                      f"{reps} launches", "peak_source": "measured bf16 cuBLAS burst"}
+
+
 def summarize_ops(per_op_ms, K, work, side_ops, hbm_peak, fp4_peak):
     """Per-op averages, throughputs and roofline fractions from the summed event times of K steps.
     `share` is an op's part of the summed main-stream (critical-path) op times; side-stream ops
@@ -532,6 +556,8 @@ def run_ours(args, rank, local_rank, world):
             e["share"] = None
             e["stream"] = "standalone, outside the step (L2 flushed before each launch, median of 20)"
             kernels[name] = e
+        kernels["kv_attention_window"] = attention_on_step_window(st, float(peaks.get("bf16_tflops",
+                                                                                    PEAK_FALLBACK["bf16_tflops"])))
     dk = kernels[dominant]
     # DRAM bytes per launch from the committed ncu summary of the dominant kernel (None when the
     # summary was taken on other kernel sources)

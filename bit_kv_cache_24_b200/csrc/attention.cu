@@ -9,26 +9,38 @@
 // k and v being exactly the values the restore produces, BF16(FP32(e2m1 * sf) * g).
 //
 // Structure (sm_100a, tcgen05): a CTA owns 256 queries of one head as two 128-row Q tiles and
-// walks the window in 128-token K/V tiles.  416 threads:
+// walks the window in 128-token K/V tiles.  512 threads, four warpgroups:
 //   warps 0-3   softmax of Q tile 0: thread = query row = tensor-memory lane
 //   warps 4-7   softmax of Q tile 1 (same lanes, its own tensor-memory columns)
 //   warps 8-11  producer: both Q tiles once, then per K/V tile the restore of one token row of K
-//               and of V into shared memory (two stages), the next tile's raw bytes already in
-//               registers
+//               and then of V into shared memory (two stages each), the next tile's raw bytes
+//               already in flight
 //   warp 12     MMA issuer (tcgen05.mma kind::f16, BF16 in, FP32 accumulate in tensor memory):
 //                 S_t = Q_t K_i^T  (A = Q_t, B = K_i: both K-major, 128-byte swizzle, in smem)
 //                 O_t += P_t V_i   (A = P_t in TENSOR memory, B = V_i: MN-major in smem)
+//   warps 13-15 idle (they complete the fourth warpgroup for the register split)
+// Each warpgroup resizes its registers first (setmaxnreg): 184 per softmax thread, 104 per
+// producer thread, 40 in the last warpgroup; per warp-scheduler slice that is 4 x 128, the 128
+// per thread the block launched with.  A softmax thread holds the tile's whole S row (128 FP32
+// values) and reads tensor memory once per tile.
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); the
 // softmax writes P_t (BF16 pairs) over the first 64 columns of S_t once it has read S_t.
 // The two Q tiles alternate: while one softmax warpgroup works on tile i, the tensor core runs
-// the other Q tile's S or P.V, and the producer restores tile i + 1.  Per Q tile the order is
-// S(i) -> softmax(i) -> P.V(i) -> S(i + 1); one thread issues all MMAs, whose execution is in
-// issue order, so S(i + 1) overwrites P(i) only after P.V(i) has read it.
+// the other Q tile's S or P.V.  Per Q tile the order is S(i) -> softmax(i) -> P.V(i) ->
+// S(i + 1); one thread issues all MMAs, whose execution is in issue order, so S(i + 1)
+// overwrites P(i) only after P.V(i) has read it.  K and V stages are released separately: a K
+// stage once both S of its tile have read it, a V stage after both P.V, so the restore of tile
+// i + 2 runs while tile i + 1 is still in flight.  A CTA whose second Q tile holds no query row
+// (the last, partial pair of rows of every head) skips that tile's MMAs and softmax; those CTAs
+// come last in the grid, after every CTA with two live tiles.
 //
 // Barriers (all waits time-bounded; a wait that gives up raises the abort flag and writes
 // NVFP4_ERR_TIMEOUT to the status word, and every role leaves its loop):
-//   kv_full[2]   count 128: the producers restored the stage (before tile 0: also both Q tiles)
-//   kv_empty[2]  count 1:   commit after the last MMA that reads the stage (P.V of Q tile 1)
+//   k_full[2]    count 128: the producers restored K of the stage (before tile 0: also both Q
+//                tiles)
+//   k_empty[2]   count 1:   commit after the last S that reads the stage
+//   v_full[2]    count 128: the producers restored V of the stage
+//   v_empty[2]   count 1:   commit after the last P.V that reads the stage
 //   s_full[t]    count 1:   commit after S_t(i) (implies P.V_t(i - 1) done, so O_t is stable)
 //   p_full[t]    count 128: softmax t wrote P_t(i) and rescaled O_t
 //   o_done[t]    count 1:   commit after the last P.V_t
@@ -45,13 +57,13 @@ namespace {
 
 constexpr int kD = 128, kBQ = 128, kBKV = 128;
 constexpr int kQTiles = 2;                         // Q tiles per CTA
-constexpr int kThreads = 416;
+constexpr int kThreads = 512;
 constexpr int kRegion = 128 * 128;                 // bytes: 128 rows x 128 B (one 64-wide d half)
 constexpr int OFF_Q = 0;                           // Q tile t at t * 2 regions
 constexpr int OFF_KV = kQTiles * 2 * kRegion;      // stage s: K at OFF_KV + s * 4R, V at + 2R
 constexpr int KV_STAGE = 4 * kRegion;
 constexpr int OFF_BAR = OFF_KV + 2 * KV_STAGE;
-constexpr int NUM_BARS = 2 + 2 + 2 + 2 + 2 + 1;
+constexpr int NUM_BARS = 2 + 2 + 2 + 2 + 2 + 2 + 2 + 1;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int kSmemBytes = OFF_MISC + 16 + 1024;
 constexpr uint32_t TMEM_COLS = 512, S_COL = 0, O_COL = 256;
@@ -209,6 +221,13 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
     return make_float2(__uint_as_float((uint32_t)d), __uint_as_float((uint32_t)(d >> 32)));
 }
 
+// max(a, b, c) in one instruction (sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -221,20 +240,29 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *sbase = smem_raw + (base - raw);
-    const uint32_t bar_kv_full = base + OFF_BAR, bar_kv_empty = bar_kv_full + 16, bar_s_full = bar_kv_empty + 16;
-    const uint32_t bar_p_full = bar_s_full + 16, bar_o_done = bar_p_full + 16, bar_drain = bar_o_done + 16;
+    const uint32_t bar_k_full = base + OFF_BAR, bar_k_empty = bar_k_full + 16;
+    const uint32_t bar_v_full = bar_k_empty + 16, bar_v_empty = bar_v_full + 16;
+    const uint32_t bar_s_full = bar_v_empty + 16, bar_p_full = bar_s_full + 16;
+    const uint32_t bar_o_done = bar_p_full + 16, bar_drain = bar_o_done + 16;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sbase + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sbase + OFF_MISC + 4);
     const int warp = __shfl_sync(0xFFFFFFFFu, (int)(threadIdx.x >> 5), 0);
     const int lane = threadIdx.x & 31;
-    const int head = blockIdx.y;
-    const int64_t q0 = (int64_t)blockIdx.x * (kQTiles * kBQ);
+    // CTAs with two live Q tiles first (head-major, so a head's CTAs run together and share its
+    // K/V in L2), the cheaper CTAs of the partial last pair of every head at the end of the grid
+    const int nfull = (int)(j.tq / (kQTiles * kBQ));
+    const int bid = blockIdx.x;
+    const int head = bid < j.heads * nfull ? bid / nfull : bid - j.heads * nfull;
+    const int64_t q0 = (int64_t)(bid < j.heads * nfull ? bid % nfull : nfull) * (kQTiles * kBQ);
     const int ntiles = (int)((j.total_tokens + kBKV - 1) / kBKV);
+    const bool q1_live = q0 + kBQ < j.tq;                // Q tile 1 holds at least one query row
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            mbar_init(bar_kv_full + 8 * i, 128);
-            mbar_init(bar_kv_empty + 8 * i, 1);
+            mbar_init(bar_k_full + 8 * i, 128);
+            mbar_init(bar_k_empty + 8 * i, 1);
+            mbar_init(bar_v_full + 8 * i, 128);
+            mbar_init(bar_v_empty + 8 * i, 1);
             mbar_init(bar_s_full + 8 * i, 1);
             mbar_init(bar_p_full + 8 * i, 128);
             mbar_init(bar_o_done + 8 * i, 1);
@@ -269,8 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
         return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
     };
 
+    // Each warpgroup first resizes its registers, out of the 128 per thread the block launched
+    // with (per warp-scheduler slice: 184 + 184 + 104 + 40 = 4 x 128), so that a softmax thread
+    // holds a whole S row.
     if (warp >= 8 && warp < 12) {
         // ------------------------------------------------------------ producer (128 threads)
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
         const int t = threadIdx.x - 256;                  // token row of the K/V tile; Q rows t, t + 128
 #pragma unroll
         for (int qt = 0; qt < kQTiles; ++qt) {
@@ -284,77 +316,82 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
                 sts_v4(qb + sw_off(t, c), v);
             }
         }
-        // the raw NVFP4 bytes of this thread's token row of a tile: loaded before the wait for the
-        // tile's stage, so the loads overlap it
+        // the raw NVFP4 bytes of this thread's token row of a tile, loaded one tile ahead
         struct RawRow {
-            uint4 ck[4], cv[4];
-            uint2 sfk, sfv;
-            float gk, gv;
-            bool live;
+            uint4 c[4];
+            uint2 sf;
+            float g;
         };
         int si = 0;
-        auto load_row = [&](int i, RawRow &rr) {
+        auto load_row = [&](int i, RawRow &rk, RawRow &rv) -> bool {
             const int64_t tok = (int64_t)i * kBKV + t;
-            rr.live = i < ntiles && tok < j.total_tokens;
-            if (!rr.live) return;
+            if (i >= ntiles || tok >= j.total_tokens) return false;
             while (si + 1 < j.nslots && tok >= j.slot[si + 1].tok_begin) ++si;
             const AttnSlot &s = j.slot[si];
             const int64_t tt = tok - s.tok_begin;
             const int64_t cb = tt * j.row_bytes + head * (kD / 2), sb = tt * j.row_sf + head * (kD / 16);
             // checked build: the token row's codes (64 B) and scales (8 B) inside the slot
-            rr.live = NVFP4_CHECKED(cb, kD / 2, s.ntok * j.row_bytes, status) &&
-                      NVFP4_CHECKED(sb, kD / 16, s.ntok * j.row_sf, status);
-            if (!rr.live) return;
-            rr.gk = *s.g_k;
-            rr.gv = *s.g_v;
-            rr.sfk = ldg_nc_v2(s.sf_k + sb);
-            rr.sfv = ldg_nc_v2(s.sf_v + sb);
+            if (!(NVFP4_CHECKED(cb, kD / 2, s.ntok * j.row_bytes, status) &&
+                  NVFP4_CHECKED(sb, kD / 16, s.ntok * j.row_sf, status)))
+                return false;
+            rk.g = *s.g_k;
+            rv.g = *s.g_v;
+            rk.sf = ldg_nc_v2(s.sf_k + sb);
+            rv.sf = ldg_nc_v2(s.sf_v + sb);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                rr.ck[q] = ldg_nc_v4(s.codes_k + cb + 16 * q);
-                rr.cv[q] = ldg_nc_v4(s.codes_v + cb + 16 * q);
+                rk.c[q] = ldg_nc_v4(s.codes_k + cb + 16 * q);
+                rv.c[q] = ldg_nc_v4(s.codes_v + cb + 16 * q);
             }
+            return true;
         };
-        bool ok = true;
-        for (int i = 0; ok && i < ntiles; ++i) {
-            const int st = i & 1;
-            RawRow cur;
-            load_row(i, cur);                             // in flight while the stage is awaited
-            if (i >= 2 && !warp_wait(bar_kv_empty + 8 * st, ((i >> 1) - 1) & 1)) { ok = false; break; }
-            const uint32_t kb = base + OFF_KV + st * KV_STAGE, vb = kb + 2 * kRegion;
-            if (cur.live) {
+        // restore one token row (128 values) into row t of a stage, or zeros past the window
+        auto store_row = [&](uint32_t sb, const RawRow &rr, bool live) {
+            if (live) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {             // 16 B of codes = 32 elements = chunks 4q..4q+3
-                    const uint32_t wk = q < 2 ? cur.sfk.x : cur.sfk.y, wv = q < 2 ? cur.sfv.x : cur.sfv.y;
-                    const uint32_t k0 = sf_f16x2(wk >> (16 * (q & 1))), k1 = sf_f16x2(wk >> (16 * (q & 1) + 8));
-                    const uint32_t v0 = sf_f16x2(wv >> (16 * (q & 1))), v1 = sf_f16x2(wv >> (16 * (q & 1) + 8));
-                    sts_v4(kb + sw_off(t, 4 * q + 0), restore8(cur.ck[q].x, k0, cur.gk));
-                    sts_v4(kb + sw_off(t, 4 * q + 1), restore8(cur.ck[q].y, k0, cur.gk));
-                    sts_v4(kb + sw_off(t, 4 * q + 2), restore8(cur.ck[q].z, k1, cur.gk));
-                    sts_v4(kb + sw_off(t, 4 * q + 3), restore8(cur.ck[q].w, k1, cur.gk));
-                    sts_v4(vb + sw_off(t, 4 * q + 0), restore8(cur.cv[q].x, v0, cur.gv));
-                    sts_v4(vb + sw_off(t, 4 * q + 1), restore8(cur.cv[q].y, v0, cur.gv));
-                    sts_v4(vb + sw_off(t, 4 * q + 2), restore8(cur.cv[q].z, v1, cur.gv));
-                    sts_v4(vb + sw_off(t, 4 * q + 3), restore8(cur.cv[q].w, v1, cur.gv));
+                    const uint32_t w = q < 2 ? rr.sf.x : rr.sf.y;
+                    const uint32_t s0 = sf_f16x2(w >> (16 * (q & 1))), s1 = sf_f16x2(w >> (16 * (q & 1) + 8));
+                    sts_v4(sb + sw_off(t, 4 * q + 0), restore8(rr.c[q].x, s0, rr.g));
+                    sts_v4(sb + sw_off(t, 4 * q + 1), restore8(rr.c[q].y, s0, rr.g));
+                    sts_v4(sb + sw_off(t, 4 * q + 2), restore8(rr.c[q].z, s1, rr.g));
+                    sts_v4(sb + sw_off(t, 4 * q + 3), restore8(rr.c[q].w, s1, rr.g));
                 }
-            } else {                                      // past the window: zero K and V rows
+            } else {
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    sts_v4(kb + sw_off(t, c), make_uint4(0, 0, 0, 0));
-                    sts_v4(vb + sw_off(t, c), make_uint4(0, 0, 0, 0));
-                }
+                for (int c = 0; c < 16; ++c) sts_v4(sb + sw_off(t, c), make_uint4(0, 0, 0, 0));
             }
+        };
+        RawRow ck, cv, nk, nv;
+        bool clive = load_row(0, ck, cv);
+        for (int i = 0; i < ntiles; ++i) {
+            const int st = i & 1;
+            const bool nlive = load_row(i + 1, nk, nv);   // in flight while tile i is restored
+            const uint32_t kb = base + OFF_KV + st * KV_STAGE, vb = kb + 2 * kRegion;
+            // K(i) into stage i % 2 once both S of tile i - 2 have read it
+            if (i >= 2 && !warp_wait(bar_k_empty + 8 * st, ((i >> 1) - 1) & 1)) break;
+            store_row(kb, ck, clive);
             fence_async_smem();                           // generic-proxy writes -> tensor core
-            mbar_arrive(bar_kv_full + 8 * st);
+            mbar_arrive(bar_k_full + 8 * st);
+            // V(i) once both P.V of tile i - 2 have read it
+            if (i >= 2 && !warp_wait(bar_v_empty + 8 * st, ((i >> 1) - 1) & 1)) break;
+            store_row(vb, cv, clive);
+            fence_async_smem();
+            mbar_arrive(bar_v_full + 8 * st);
+            ck = nk;
+            cv = nv;
+            clive = nlive;
         }
-    } else if (warp == 12) {
+    } else if (warp >= 12) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+        if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer (whole warp)
         bool ok = true, issued = false;
         // S_t(i) = Q_t K_i^T into S_t; the stage's K is read by both Q tiles
         auto issue_s = [&](int qt, int i) {
             const uint64_t qdesc = kmajor_desc(base + OFF_Q + qt * 2 * kRegion);
             const uint64_t kdesc = kmajor_desc(base + OFF_KV + (i & 1) * KV_STAGE);
-#pragma unroll
+#pragma unroll 1
             for (int kk = 0; kk < kD / 16; ++kk) {
                 // K step kk: region kk / 4, 32 bytes per step inside the 128-byte row
                 const uint64_t off = (uint64_t)((kk >> 2) * (kRegion >> 4) + 2 * (kk & 3));
@@ -366,50 +403,70 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
         // O_t += P_t(i) V_i: A = P_t (BF16 pairs in the first 64 columns of S_t), B = V_i
         auto issue_pv = [&](int qt, int i) {
             const uint32_t vbase = base + OFF_KV + (i & 1) * KV_STAGE + 2 * kRegion;
-#pragma unroll
+#pragma unroll 1
             for (int kt = 0; kt < kBKV / 16; ++kt)
                 tc_mma_ts(tmem + O_COL + 128 * qt, tmem + S_COL + 128 * qt + 8 * kt, mnmajor_desc(vbase + 2048 * kt),
                           kIdescPV, (i | kt) != 0);
         };
-        if (ntiles > 0 && warp_wait(bar_kv_full, 0)) {
+        auto wait_k = [&](int i) -> bool {
+            if (!warp_wait(bar_k_full + 8 * (i & 1), (i >> 1) & 1)) return false;
             tc_fence_after();
-            issue_s(0, 0);
-            issue_s(1, 0);
+            return true;
+        };
+        // S of both Q tiles, then K's stage goes back to the producer
+        auto issue_s_pair = [&](int i) {
+            issue_s(0, i);
+            if (q1_live) issue_s(1, i);
+            tc_commit(bar_k_empty + 8 * (i & 1));
+        };
+        if (ntiles > 0 && wait_k(0)) {
+            issue_s_pair(0);
         } else {
             ok = false;
         }
         for (int i = 0; ok && i < ntiles; ++i) {
             const bool more = i + 1 < ntiles;
-            // Q tile 0: P.V(i), then S(i + 1) as soon as K(i + 1) is restored
-            if (!warp_wait(bar_p_full, i & 1)) { ok = false; break; }
+            // Q tile 0: P.V(i) once its P and V(i) are in place
+            if (!warp_wait(bar_p_full, i & 1) || !warp_wait(bar_v_full + 8 * (i & 1), (i >> 1) & 1)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
             issue_pv(0, i);
+            if (!q1_live) tc_commit(bar_v_empty + 8 * (i & 1));
             if (!more) tc_commit(bar_o_done);
+            // S_0(i + 1) as soon as K(i + 1) is restored; S_1(i + 1) after P.V_1(i) (P_1 lives in S_1)
             if (more) {
-                if (!warp_wait(bar_kv_full + 8 * ((i + 1) & 1), ((i + 1) >> 1) & 1)) { ok = false; break; }
-                tc_fence_after();
+                if (!wait_k(i + 1)) { ok = false; break; }
                 issue_s(0, i + 1);
             }
-            // Q tile 1: P.V(i) frees stage i % 2, then S(i + 1)
-            if (!warp_wait(bar_p_full + 8, i & 1)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(1, i);
-            tc_commit(bar_kv_empty + 8 * (i & 1));
-            if (!more) tc_commit(bar_o_done + 8);
-            if (more) issue_s(1, i + 1);
+            if (q1_live) {
+                if (!warp_wait(bar_p_full + 8, i & 1)) { ok = false; break; }
+                tc_fence_after();
+                issue_pv(1, i);
+                tc_commit(bar_v_empty + 8 * (i & 1));
+                if (!more) tc_commit(bar_o_done + 8);
+                if (more) issue_s(1, i + 1);
+            }
+            if (more) tc_commit(bar_k_empty + 8 * ((i + 1) & 1));
         }
         if (issued) {
             tc_commit(bar_drain);
             if (lane == 0 && !mbar_wait_bounded(bar_drain, 0, nullptr, kWaitLimitNs)) give_up();
         }
         __syncwarp();
-    } else if (warp < 8) {
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
+        if (warp < 4 || q1_live) {
         // ------------------------------------------------------------ softmax + epilogue
         const int qt = warp >> 2;                         // Q tile of this warpgroup
         const int r = threadIdx.x & 127;                  // query row = tensor-memory lane
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const uint32_t scol = lane_base + S_COL + 128 * qt, ocol = lane_base + O_COL + 128 * qt;
         const uint32_t s_full = bar_s_full + 8 * qt, p_full = bar_p_full + 8 * qt;
+        const float c2 = j.scale_log2;
+        const bool pos = c2 >= 0.0f;
         float m = -INFINITY, l = 0.0f;
         bool ok = true;
         for (int i = 0; ok && i < ntiles; ++i) {
@@ -417,85 +474,81 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
             tc_fence_after();
             const int64_t t0 = (int64_t)i * kBKV;
             const bool full = t0 + kBKV <= j.total_tokens;
-            // pass 1: the row maximum of the tile's raw scores (tokens past the window excluded);
-            // scaling it afterwards gives the maximum of the scaled scores exactly (rounding is
-            // monotone), for a positive scale; a negative scale takes the minimum instead
-            const float c2 = j.scale_log2;
-            const bool pos = c2 >= 0.0f;
+            // the tile's 128 raw scores of this row, in one batch of tensor-memory loads
+            uint32_t s[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc_ld32_nowait(scol + 32 * c, s[c]);
+            tc_wait_ld();
+            // the row maximum of the raw scores (tokens past the window excluded); scaling it
+            // afterwards gives the maximum of the scaled scores exactly (rounding is monotone), for a
+            // positive scale; a negative scale takes the minimum instead
             float xm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int c = 0; c < 4; c += 2) {
-                uint32_t v0[32], v1[32];
-                tc_ld32_nowait(scol + 32 * c, v0);
-                tc_ld32_nowait(scol + 32 * c + 32, v1);
-                tc_wait_ld();
-                if (full && pos) {
+            if (full && pos) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        xm[e & 3] = fmaxf(xm[e & 3], __uint_as_float(v0[e]));
-                        xm[e & 3] = fmaxf(xm[e & 3], __uint_as_float(v1[e]));
-                    }
-                } else {
+                for (int c = 0; c < 4; ++c)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
+                    for (int e = 0; e < 32; e += 2)
+                        xm[(e >> 1) & 3] = fmax3(xm[(e >> 1) & 3], __uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1]));
+            } else {
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
                         if (t0 + 32 * c + e < j.total_tokens)
-                            xm[e & 3] = fmaxf(xm[e & 3], pos ? __uint_as_float(v0[e]) : -__uint_as_float(v0[e]));
-                        if (t0 + 32 * c + 32 + e < j.total_tokens)
-                            xm[e & 3] = fmaxf(xm[e & 3], pos ? __uint_as_float(v1[e]) : -__uint_as_float(v1[e]));
-                    }
-                }
+                            xm[e & 3] = fmaxf(xm[e & 3], pos ? __uint_as_float(s[c][e]) : -__uint_as_float(s[c][e]));
             }
             const float xr = fmaxf(fmaxf(xm[0], xm[1]), fmaxf(xm[2], xm[3]));
             const float x = xr == -INFINITY ? -INFINITY : (pos ? xr * c2 : -xr * c2);
             const float mn = fmaxf(m, x);
             const float b = mn == -INFINITY ? 0.0f : mn;
             const float alpha = ex2(m - b);
-            // O_t is stable here (s_full(i) implies P.V(i - 1) done): rescale it when any row of
-            // the warp moved its maximum (tcgen05.ld/st are warp-wide)
-            if (i > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t v[32];
-                    tc_ld32_nowait(ocol + 32 * c, v);
-                    tc_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-                    tc_st32(ocol + 32 * c, v);
-                }
-            }
-            // pass 2: P = 2^(s * c2 - b) (BF16 pairs) and its row sum, paired FP32 arithmetic; in
-            // two halves of 64 tokens, each written over S columns already read (P half h to
-            // columns [32h, 32h + 32), from S columns [64h, 64h + 64))
+            // P = 2^(s * c2 - b) (BF16 pairs) and its row sum, paired FP32 arithmetic; P's 64 words go
+            // to S columns [0, 64), already read
             float2 sum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-#pragma unroll 1
+#pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t p[32];
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c = 2 * hh + cc;
-                    uint32_t v[32];
-                    tc_ld32_nowait(scol + 32 * c, v);
-                    tc_wait_ld();
                     if (full) {
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const float2 t = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), c2, -b);
-                            const float2 pp = make_float2(ex2(t.x), ex2(t.y));
+                            const float2 tv = fma2(make_float2(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), c2, -b);
+                            const float2 pp = make_float2(ex2(tv.x), ex2(tv.y));
                             sum2[(e >> 1) & 1] = add2(sum2[(e >> 1) & 1], pp);
                             p[16 * cc + e / 2] = bf16x2(pp.x, pp.y);
                         }
                     } else {
 #pragma unroll
                         for (int e = 0; e < 32; e += 2) {
-                            const float2 t = fma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), c2, -b);
-                            const float p0 = t0 + 32 * c + e < j.total_tokens ? ex2(t.x) : 0.0f;
-                            const float p1 = t0 + 32 * c + e + 1 < j.total_tokens ? ex2(t.y) : 0.0f;
+                            const float2 tv = fma2(make_float2(__uint_as_float(s[c][e]), __uint_as_float(s[c][e + 1])), c2, -b);
+                            const float p0 = t0 + 32 * c + e < j.total_tokens ? ex2(tv.x) : 0.0f;
+                            const float p1 = t0 + 32 * c + e + 1 < j.total_tokens ? ex2(tv.y) : 0.0f;
                             sum2[(e >> 1) & 1] = add2(sum2[(e >> 1) & 1], make_float2(p0, p1));
                             p[16 * cc + e / 2] = bf16x2(p0, p1);
                         }
                     }
                 }
                 tc_st32(scol + 32 * hh, p);
+            }
+            // O_t is stable here (s_full(i) implies P.V(i - 1) done; P.V(i) waits for p_full): rescale
+            // it when any row of the warp moved its maximum (tcgen05.ld/st are warp-wide)
+            if (i > 0 && __any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+#pragma unroll 1
+                for (int c = 0; c < 4; c += 2) {
+                    uint32_t v0[32], v1[32];
+                    tc_ld32_nowait(ocol + 32 * c, v0);
+                    tc_ld32_nowait(ocol + 32 * c + 32, v1);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
+                        v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
+                    }
+                    tc_st32(ocol + 32 * c, v0);
+                    tc_st32(ocol + 32 * c + 32, v1);
+                }
             }
             const float sum = (sum2[0].x + sum2[0].y) + (sum2[1].x + sum2[1].y);
             l = l * alpha + sum;
@@ -527,8 +580,8 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
                 }
             }
         }
+        }
     }
-
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -550,7 +603,7 @@ cudaError_t launch_kv_attention(const AttnJob &j, int32_t *status, cudaStream_t 
         if (e != cudaSuccess) return e;
         attr_set[dev].store(true, std::memory_order_release);
     }
-    const dim3 grid((unsigned)ceil_div(j.tq, kQTiles * kBQ), (unsigned)j.heads);
+    const dim3 grid((unsigned)(ceil_div(j.tq, kQTiles * kBQ) * j.heads));
     return launch_pdl(kv_attention_kernel, grid, dim3(kThreads), kSmemBytes, s, j, status);
 }
 
