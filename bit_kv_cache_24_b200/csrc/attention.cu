@@ -287,14 +287,11 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
         *abort_flag = 1;
         set_status(status, NVFP4_ERR_TIMEOUT);
     };
-    // lane 0 of a converged warp waits and broadcasts the outcome, so no warp diverges on it
+    // every lane of a converged warp tests the phase (a vote decides), so no warp diverges on it
     auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
-        bool ok = true;
-        if (lane == 0) {
-            ok = mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs);
-            if (!ok) give_up();
-        }
-        return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        const bool ok = mbar_wait_warp(bar, parity, abort_flag, kWaitLimitNs);
+        if (!ok && lane == 0) give_up();
+        return ok;
     };
 
     // Each warpgroup first resizes its registers, out of the 128 per thread the block launched

@@ -316,6 +316,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// Warp-wide form of mbar_wait_bounded, called by all 32 lanes of a converged warp.  Every lane
+// tests the phase in the same instruction and the outcome is taken with a vote, so a wait on a
+// phase that is already complete costs no more than any other instruction; only an open phase
+// falls through to the sleeping, time-bounded loop, whose decisions are voted too (warp-uniform).
+// (A lane-0 wait followed by a shuffle broadcast cost ~110-170 cycles per call on a complete
+// phase, and an MMA-issuing warp pays that between every group of MMAs.)
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const volatile int *abort,
+                                               uint64_t limit_ns) {
+    if (__any_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity))) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (__any_sync(0xFFFFFFFFu, mbar_try_wait_sleep(bar, parity, 20000u))) return true;
+        if (__any_sync(0xFFFFFFFFu, (abort && *abort) || globaltimer_ns() - t0 > limit_ns)) return false;
+    }
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
 }

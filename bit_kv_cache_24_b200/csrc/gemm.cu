@@ -202,12 +202,9 @@ nvfp4_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_consta
     };
     // lane 0 of the warp waits; the outcome is broadcast so the warp never diverges on it
     auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
-        bool ok = true;
-        if (lane == 0) {
-            ok = mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs);
-            if (!ok) give_up();
-        }
-        return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        const bool ok = mbar_wait_warp(bar, parity, abort_flag, kWaitLimitNs);
+        if (!ok && lane == 0) give_up();
+        return ok;
     };
 
     if (warp == 0) {

@@ -245,12 +245,9 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
         set_status(args.status, NVFP4_ERR_TIMEOUT);
     };
     auto warp_wait = [&](uint32_t bar, uint32_t parity) -> bool {
-        bool ok = true;
-        if (lane == 0) {
-            ok = mbar_wait_bounded(bar, parity, abort_flag, kWaitLimitNs);
-            if (!ok) give_up();
-        }
-        return __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+        const bool ok = mbar_wait_warp(bar, parity, abort_flag, kWaitLimitNs);
+        if (!ok && lane == 0) give_up();
+        return ok;
     };
 
     if (warp == 0) {
@@ -313,12 +310,7 @@ nvfp4_gemm_2sm_kernel(const __grid_constant__ Maps maps, const __grid_constant__
         uint32_t stage = 0, phase = 0, acc_phase = 0;
         bool ok = true, issued = false;
         for (int t = cluster; ok && t < num_tiles; t += nclusters) {
-            bool got = true;
-            if (lane == 0) {
-                got = mbar_wait_bounded(bar_tmem_empty, acc_phase ^ 1, abort_flag, kWaitLimitNs);
-                if (!got) give_up();
-            }
-            if (!__shfl_sync(0xFFFFFFFFu, got ? 1 : 0, 0)) break;
+            if (!warp_wait(bar_tmem_empty, acc_phase ^ 1)) break;
             tc_fence_after();
             for (int kt = 0; kt < nkt; ++kt) {
                 if (!warp_wait(bar_full + 8 * stage, phase) || !warp_wait(bar_sf + 8 * stage, phase)) {
