@@ -65,6 +65,9 @@ def parse_args(argv=None):
     p.add_argument("--no-large-gemms", action="store_true",
                    help="skip the standalone FFN and training-shape GEMM timings of the default run")
     p.add_argument("--cpu-seconds", type=float, default=15.0)
+    p.add_argument("--attn-slots", type=int, default=SLOTS,
+                   help="--op attention: cache slots in the window (default 12 = 56160 tokens; 1 gives the "
+                        "small case used for ncu captures)")
     p.add_argument("--op", choices=["step", "attention", "appends", "kernels"], default="step",
                    help="step: the QKV chunk step (default); attention: kv_attention over the step's KV "
                         "window; appends: one chunk's KV append into all 30 layers, as a CUDA graph; "
@@ -683,15 +686,19 @@ def run_attention(args, rank, local_rank, world):
     dist = init_dist(world, "nccl")
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cache = nv.KVCache(1, HEADS, HEAD_DIM, SLOTS, M_TOK, dev)
-    for s in range(SLOTS):
+    nslots = args.attn_slots
+    if not 1 <= nslots <= SLOTS:
+        raise SystemExit(f"--attn-slots must be in [1, {SLOTS}]")
+    attn_flop = ATTN_FLOP * nslots / SLOTS
+    cache = nv.KVCache(1, HEADS, HEAD_DIM, nslots, M_TOK, dev)
+    for s in range(nslots):
         k, v = synth.kv_chunk(0, s)
         nv.kv_quant_append(cache, 0, s, k.to(dev), v.to(dev))
     q_host = synth.normal(21, 0, (M_TOK, HEADS, HEAD_DIM)).pin_memory()
     q = q_host.to(dev)
     o = torch.empty_like(q)
     o_host = torch.empty_like(q_host).pin_memory()
-    slots, scale = list(range(SLOTS)), 1.0 / math.sqrt(HEAD_DIM)
+    slots, scale = list(range(nslots)), 1.0 / math.sqrt(HEAD_DIM)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
         nv.kv_attention(cache, 0, slots, q, scale, out=o)
@@ -708,7 +715,7 @@ def run_attention(args, rank, local_rank, world):
     torch.cuda.synchronize()
     clk = clocks.stop()
     max_s = reduce_max(ev[0].elapsed_time(ev[1]) / 1e3, dist, dev)
-    value = aggregate(ATTN_FLOP * K / 1e12, world, max_s)
+    value = aggregate(attn_flop * K / 1e12, world, max_s)
 
     # end to end through the public call: q in from pinned host memory, O back out, every step
     E = max(3, min(K, 20))
@@ -725,7 +732,7 @@ def run_attention(args, rank, local_rank, world):
 
     peaks, src = load_peaks()
     peak = float(peaks.get("bf16_tflops", PEAK_FALLBACK["bf16_tflops"]))
-    ach = ATTN_FLOP / (max_s / K) / 1e12
+    ach = attn_flop / (max_s / K) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = attention_cpu_baseline(args.cpu_seconds)
@@ -735,16 +742,18 @@ def run_attention(args, rank, local_rank, world):
         "ms_per_step": round(max_s * 1e3 / K, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4 K/V (e2m1 x e4m3/16) -> bf16 mma, fp32 acc -> bf16",
         "data": "synthetic (seeded; K/V of the KV workload, q ~ N(0,1))",
-        "config": {"workload": "kv_attention: 4680 queries x 24 heads x 128 over the 12-slot NVFP4 window "
-                               "(56160 tokens), no mask", "global_batch": M_TOK * world, "seq_len": SLOTS * M_TOK,
+        "config": {"workload": f"kv_attention: 4680 queries x 24 heads x 128 over the {nslots}-slot NVFP4 window "
+                               f"({nslots * M_TOK} tokens), no mask", "global_batch": M_TOK * world,
+                   "seq_len": nslots * M_TOK,
                    "parallelism": f"replicas x{world}",
-                   "l2": "the window's NVFP4 K/V (194 MB) exceeds the 126 MB L2"},
+                   "l2": f"the window's NVFP4 K/V ({nslots * 16.2:.0f} MB) "
+                         + ("exceeds the 126 MB L2" if nslots * 16.2 > 126 else "fits in the 126 MB L2")},
         "gpu_launches": K,
         "roofline": {"kernel": "kv_attention_kernel", "bound": "tensor", "achieved": round(ach, 1),
                      "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(ach / peak, 4), "traffic": None,
                      "peak_source": f"{src} (bf16 cuBLAS burst)"},
         "clocks": clk,
-        "e2e": {"value": round(aggregate(ATTN_FLOP * E / 1e12, world, e2e_s), 2), "unit": "TFLOP/s",
+        "e2e": {"value": round(aggregate(attn_flop * E / 1e12, world, e2e_s), 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes, "steps": E},
     }
     if cpu is not None:
