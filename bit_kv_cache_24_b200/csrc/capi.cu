@@ -268,6 +268,7 @@ nvfp4_status nvfp4_quantize(const void *x_bf16, int64_t M, int64_t K, int64_t ld
     } else {
         e = launch_amax(jobs, dev_status, nullptr, s);
         if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+        j.x_early = 1;                                    // the amax pass read x after its wait
     }
     if (e == cudaSuccess && row_out) {
         j.codes = row_out->codes;
@@ -448,6 +449,7 @@ nvfp4_status kv_quant_append_amax(nvfp4_kv_cache *cache, int32_t layer, int32_t 
     if (!amax_kv) {
         e = launch_amax(jobs, dev_status, nullptr, s);
         if (e == cudaSuccess) e = launch_scale_record(rj, dev_status, s);
+        for (int i = 0; i < 2; ++i) jobs.job[i].x_early = 1;   // the amax pass read x after its wait
     }
     if (e == cudaSuccess) e = launch_quantize_rows(jobs, s);
     if (e != cudaSuccess) return cuda_fail(e, "kv_quant_append");

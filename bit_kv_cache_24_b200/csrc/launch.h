@@ -40,6 +40,10 @@ struct RowJob {
     const float *amax_in;
     float *g_out[2];
     int32_t report_record;
+    // Set only when x was complete before this job's own amax pass read it (amax pass, record
+    // kernel, then this pass): the row pass then loads x before its dependency wait, overlapping
+    // the loads with the record kernel, and waits only before reading the record.
+    int32_t x_early;
     int32_t *status;
     // buffer extents for the checked build (see NVFP4_CHECKED): elements of x from its start,
     // bytes of codes and of sf

@@ -277,9 +277,12 @@ __global__ void __launch_bounds__(kThreads) scale_record_kernel(const __grid_con
 // (to a multiple of 64) of the tensor-core layout.
 template <bool kV8, bool kMma>
 __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_constant__ RowJobs jobs) {
-    griddep_wait();
-    griddep_launch_dependents();
     const RowJob &j = jobs.job[blockIdx.y];
+    const bool early = j.x_early != 0;                     // x complete before the amax pass read it
+    if (!early) {
+        griddep_wait();
+        griddep_launch_dependents();
+    }
     __shared__ SmemRecord rec;
     const uint32_t rows = (uint32_t)j.rows;
     const uint32_t nb = (uint32_t)(j.cols >> 4);            // 16-blocks per row
@@ -310,6 +313,10 @@ __global__ void __launch_bounds__(kThreads) quantize_rows_kernel(const __grid_co
 #pragma unroll
             for (int i = 0; i < 8; ++i) w[b][i] = 0;
         }
+    }
+    if (early) {                                          // the record kernel's output from here on
+        griddep_wait();
+        griddep_launch_dependents();
     }
     if (j.amax_in)
         build_record(*j.amax_in, rec, j.report_record && blockIdx.x == 0, j.g_out[0], j.g_out[1], j.status);
