@@ -9,20 +9,20 @@
 // k and v being exactly the values the restore produces, BF16(FP32(e2m1 * sf) * g).
 //
 // Structure (sm_100a, tcgen05): a CTA owns 256 queries of one head as two 128-row Q tiles and
-// walks the window in 128-token K/V tiles.  512 threads, four warpgroups:
+// walks the window in 128-token K/V tiles.  640 threads, five warpgroups:
 //   warps 0-3   softmax of Q tile 0: thread = query row = tensor-memory lane
 //   warps 4-7   softmax of Q tile 1 (same lanes, its own tensor-memory columns)
-//   warps 8-11  producer: both Q tiles once, then per K/V tile the restore of one token row of K
-//               and then of V into shared memory (two stages each), the next tile's raw bytes
-//               already in flight
-//   warp 12     MMA issuer (tcgen05.mma kind::f16, BF16 in, FP32 accumulate in tensor memory):
+//   warps 8-11  K producer: both Q tiles once, then per K/V tile the restore of one token row
+//               of K into shared memory (two stages)
+//   warps 12-15 V producer: the same for V (two stages)
+//   warp 16     MMA issuer (tcgen05.mma kind::f16, BF16 in, FP32 accumulate in tensor memory):
 //                 S_t = Q_t K_i^T  (A = Q_t, B = K_i: both K-major, 128-byte swizzle, in smem)
 //                 O_t += P_t V_i   (A = P_t in TENSOR memory, B = V_i: MN-major in smem)
-//   warps 13-15 idle (they complete the fourth warpgroup for the register split)
-// Each warpgroup resizes its registers first (setmaxnreg): 184 per softmax thread, 104 per
-// producer thread, 40 in the last warpgroup; per warp-scheduler slice that is 4 x 128, the 128
-// per thread the block launched with.  A softmax thread holds the tile's whole S row (128 FP32
-// values) and reads tensor memory once per tile.
+//   warps 17-19 idle (they complete the fifth warpgroup for the register split)
+// Each warpgroup resizes its registers first (setmaxnreg): 176 per softmax thread, 40 per
+// producer thread, 48 in the last warpgroup; per warp-scheduler slice that is 5 x 96, the 96 per
+// thread the block launched with (the launcher checks the 96).  A softmax thread holds the
+// tile's whole S row (128 FP32 values) and reads tensor memory once per tile.
 // Tensor memory (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512); the
 // softmax writes P_t (BF16 pairs) over the first 64 columns of S_t once it has read S_t.
 // The two Q tiles alternate: while one softmax warpgroup works on tile i, the tensor core runs
@@ -36,10 +36,10 @@
 //
 // Barriers (all waits time-bounded; a wait that gives up raises the abort flag and writes
 // NVFP4_ERR_TIMEOUT to the status word, and every role leaves its loop):
-//   k_full[2]    count 128: the producers restored K of the stage (before tile 0: also both Q
+//   k_full[2]    count 128: the K producers restored K of the stage (before tile 0: also both Q
 //                tiles)
 //   k_empty[2]   count 1:   commit after the last S that reads the stage
-//   v_full[2]    count 128: the producers restored V of the stage
+//   v_full[2]    count 128: the V producers restored V of the stage
 //   v_empty[2]   count 1:   commit after the last P.V that reads the stage
 //   s_full[t]    count 1:   commit after S_t(i) (implies P.V_t(i - 1) done, so O_t is stable)
 //   p_full[t]    count 128: softmax t wrote P_t(i) and rescaled O_t
@@ -57,7 +57,14 @@ namespace {
 
 constexpr int kD = 128, kBQ = 128, kBKV = 128;
 constexpr int kQTiles = 2;                         // Q tiles per CTA
-constexpr int kThreads = 512;
+constexpr int kThreads = 640;
+constexpr int kMmaWarp = 16;
+// registers per thread at launch (the most __launch_bounds__(kThreads, 1) allows) and the
+// warpgroups' shares after setmaxnreg: two softmax, two producer, one MMA warpgroup
+constexpr int kLaunchRegs = (65536 / kThreads) & ~7;
+constexpr int kRegsSoftmax = 176, kRegsProducer = 40, kRegsMma = 48;
+static_assert(2 * kRegsSoftmax + 2 * kRegsProducer + kRegsMma == 5 * kLaunchRegs,
+              "the register split must add up to the launch's registers");
 constexpr int kRegion = 128 * 128;                 // bytes: 128 rows x 128 B (one 64-wide d half)
 constexpr int OFF_Q = 0;                           // Q tile t at t * 2 regions
 constexpr int OFF_KV = kQTiles * 2 * kRegion;      // stage s: K at OFF_KV + s * 4R, V at + 2R
@@ -271,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (warp == 12) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      :: "r"(smem_addr(tmem_slot)), "r"(TMEM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -294,33 +301,37 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
         return ok;
     };
 
-    // Each warpgroup first resizes its registers, out of the 128 per thread the block launched
-    // with (per warp-scheduler slice: 184 + 184 + 104 + 40 = 4 x 128), so that a softmax thread
-    // holds a whole S row.
-    if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------------------ producer (128 threads)
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
-        const int t = threadIdx.x - 256;                  // token row of the K/V tile; Q rows t, t + 128
+    // Each warpgroup first resizes its registers, out of the 96 per thread the block launched with
+    // (per warp-scheduler slice: 2 x 176 + 2 x 40 + 48 = 5 x 96), so that a softmax thread holds a
+    // whole S row.
+    if (warp >= 8 && warp < 16) {
+        // ------------------------------------------------------------ producers (K: warps 8-11,
+        // V: warps 12-15), one token row of the tile per thread
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsProducer) : "memory");
+        const bool is_v = warp >= 12;
+        const int t = threadIdx.x & 127;
+        if (!is_v) {                                      // both Q tiles, before K(0)
+#pragma unroll 1
+            for (int qt = 0; qt < kQTiles; ++qt) {
+                const int64_t r = q0 + qt * kBQ + t;
+                const uint16_t *src = j.q + r * j.ldq + head * kD;
+                const uint32_t qb = base + OFF_Q + qt * 2 * kRegion;
 #pragma unroll
-        for (int qt = 0; qt < kQTiles; ++qt) {
-            const int64_t r = q0 + qt * kBQ + t;
-            const uint16_t *src = j.q + r * j.ldq + head * kD;
-            const uint32_t qb = base + OFF_Q + qt * 2 * kRegion;
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const uint4 v = r < j.tq && NVFP4_CHECKED(r * j.ldq + head * kD + 8 * c, 8, j.q_elems, status)
-                                    ? ldg_nc_v4(src + 8 * c) : make_uint4(0, 0, 0, 0);
-                sts_v4(qb + sw_off(t, c), v);
+                for (int c = 0; c < 16; ++c) {
+                    const uint4 v = r < j.tq && NVFP4_CHECKED(r * j.ldq + head * kD + 8 * c, 8, j.q_elems, status)
+                                        ? ldg_nc_v4(src + 8 * c) : make_uint4(0, 0, 0, 0);
+                    sts_v4(qb + sw_off(t, c), v);
+                }
             }
         }
-        // the raw NVFP4 bytes of this thread's token row of a tile, loaded one tile ahead
+        // the raw NVFP4 bytes of this thread's token row of a tile
         struct RawRow {
             uint4 c[4];
             uint2 sf;
             float g;
         };
         int si = 0;
-        auto load_row = [&](int i, RawRow &rk, RawRow &rv) -> bool {
+        auto load_row = [&](int i, RawRow &rr) -> bool {
             const int64_t tok = (int64_t)i * kBKV + t;
             if (i >= ntiles || tok >= j.total_tokens) return false;
             while (si + 1 < j.nslots && tok >= j.slot[si + 1].tok_begin) ++si;
@@ -331,57 +342,42 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
             if (!(NVFP4_CHECKED(cb, kD / 2, s.ntok * j.row_bytes, status) &&
                   NVFP4_CHECKED(sb, kD / 16, s.ntok * j.row_sf, status)))
                 return false;
-            rk.g = *s.g_k;
-            rv.g = *s.g_v;
-            rk.sf = ldg_nc_v2(s.sf_k + sb);
-            rv.sf = ldg_nc_v2(s.sf_v + sb);
+            const uint8_t *codes = is_v ? s.codes_v : s.codes_k;
+            rr.g = is_v ? *s.g_v : *s.g_k;
+            rr.sf = ldg_nc_v2((is_v ? s.sf_v : s.sf_k) + sb);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                rk.c[q] = ldg_nc_v4(s.codes_k + cb + 16 * q);
-                rv.c[q] = ldg_nc_v4(s.codes_v + cb + 16 * q);
-            }
+            for (int q = 0; q < 4; ++q) rr.c[q] = ldg_nc_v4(codes + cb + 16 * q);
             return true;
         };
-        // restore one token row (128 values) into row t of a stage, or zeros past the window
-        auto store_row = [&](uint32_t sb, const RawRow &rr, bool live) {
-            if (live) {
+        const uint32_t full = is_v ? bar_v_full : bar_k_full, empty = is_v ? bar_v_empty : bar_k_empty;
+        const uint32_t off = is_v ? 2 * kRegion : 0;
+        RawRow cur;
+        for (int i = 0; i < ntiles; ++i) {
+            const int st = i & 1;
+            const bool clive = load_row(i, cur);          // in flight while the stage is awaited
+            const uint32_t sb = base + OFF_KV + st * KV_STAGE + off;
+            // the stage once the MMAs of tile i - 2 that read it (both S, or both P.V) are done
+            if (i >= 2 && !warp_wait(empty + 8 * st, ((i >> 1) - 1) & 1)) break;
+            if (clive) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {             // 16 B of codes = 32 elements = chunks 4q..4q+3
-                    const uint32_t w = q < 2 ? rr.sf.x : rr.sf.y;
+                    const uint32_t w = q < 2 ? cur.sf.x : cur.sf.y;
                     const uint32_t s0 = sf_f16x2(w >> (16 * (q & 1))), s1 = sf_f16x2(w >> (16 * (q & 1) + 8));
-                    sts_v4(sb + sw_off(t, 4 * q + 0), restore8(rr.c[q].x, s0, rr.g));
-                    sts_v4(sb + sw_off(t, 4 * q + 1), restore8(rr.c[q].y, s0, rr.g));
-                    sts_v4(sb + sw_off(t, 4 * q + 2), restore8(rr.c[q].z, s1, rr.g));
-                    sts_v4(sb + sw_off(t, 4 * q + 3), restore8(rr.c[q].w, s1, rr.g));
+                    sts_v4(sb + sw_off(t, 4 * q + 0), restore8(cur.c[q].x, s0, cur.g));
+                    sts_v4(sb + sw_off(t, 4 * q + 1), restore8(cur.c[q].y, s0, cur.g));
+                    sts_v4(sb + sw_off(t, 4 * q + 2), restore8(cur.c[q].z, s1, cur.g));
+                    sts_v4(sb + sw_off(t, 4 * q + 3), restore8(cur.c[q].w, s1, cur.g));
                 }
-            } else {
+            } else {                                      // past the window: zero rows
 #pragma unroll
                 for (int c = 0; c < 16; ++c) sts_v4(sb + sw_off(t, c), make_uint4(0, 0, 0, 0));
             }
-        };
-        RawRow ck, cv, nk, nv;
-        bool clive = load_row(0, ck, cv);
-        for (int i = 0; i < ntiles; ++i) {
-            const int st = i & 1;
-            const bool nlive = load_row(i + 1, nk, nv);   // in flight while tile i is restored
-            const uint32_t kb = base + OFF_KV + st * KV_STAGE, vb = kb + 2 * kRegion;
-            // K(i) into stage i % 2 once both S of tile i - 2 have read it
-            if (i >= 2 && !warp_wait(bar_k_empty + 8 * st, ((i >> 1) - 1) & 1)) break;
-            store_row(kb, ck, clive);
             fence_async_smem();                           // generic-proxy writes -> tensor core
-            mbar_arrive(bar_k_full + 8 * st);
-            // V(i) once both P.V of tile i - 2 have read it
-            if (i >= 2 && !warp_wait(bar_v_empty + 8 * st, ((i >> 1) - 1) & 1)) break;
-            store_row(vb, cv, clive);
-            fence_async_smem();
-            mbar_arrive(bar_v_full + 8 * st);
-            ck = nk;
-            cv = nv;
-            clive = nlive;
+            mbar_arrive(full + 8 * st);
         }
-    } else if (warp >= 12) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
-        if (warp == 12) {
+    } else if (warp >= 16) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(kRegsMma) : "memory");
+        if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer (whole warp)
         bool ok = true, issued = false;
         // S_t(i) = Q_t K_i^T into S_t; the stage's K is read by both Q tiles
@@ -454,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
         __syncwarp();
         }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(kRegsSoftmax) : "memory");
         if (warp < 4 || q1_live) {
         // ------------------------------------------------------------ softmax + epilogue
         const int qt = warp >> 2;                         // Q tile of this warpgroup
@@ -582,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) kv_attention_kernel(const __grid_
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 12) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMEM_COLS) : "memory");
     }
 }
@@ -598,6 +594,12 @@ cudaError_t launch_kv_attention(const AttnJob &j, int32_t *status, cudaStream_t 
     if (dev >= 0 && dev < 64 && !attr_set[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(kv_attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
+        // setmaxnreg.inc draws on the registers the block launched with: launched with fewer
+        // than the split assumes, the softmax warpgroups would wait for registers forever
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, kv_attention_kernel);
+        if (e != cudaSuccess) return e;
+        if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
         attr_set[dev].store(true, std::memory_order_release);
     }
     const dim3 grid((unsigned)(ceil_div(j.tq, kQTiles * kBQ) * j.heads));

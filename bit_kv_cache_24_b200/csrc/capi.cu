@@ -356,6 +356,7 @@ nvfp4_status nvfp4_gemm_colamax(const nvfp4_tensor *A, const nvfp4_tensor *B, co
     if (!amax_out || !ws || group_cols <= 0 || ws_bytes < nvfp4_gemm_colamax_workspace(M, N))
         return NVFP4_ERR_INVALID_ARG;
     if ((group_cols & 255) || N % group_cols || !aligned16(ws)) return NVFP4_ERR_UNSUPPORTED;
+    if (ceil_div(M, 32) * (group_cols / 128) >= (int64_t(1) << 31)) return NVFP4_ERR_UNSUPPORTED;   // finish indexing
     st = check_device();
     if (st != NVFP4_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

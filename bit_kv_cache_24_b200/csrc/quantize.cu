@@ -197,25 +197,25 @@ __global__ void __launch_bounds__(kThreads) colamax_finish_kernel(const uint32_t
     griddep_wait();
     griddep_launch_dependents();
     __shared__ uint32_t red[kWarps];
-    constexpr int kRowsInFlight = 8;
+    // the group's rows32 x cpg partials as one flat range: each thread issues all of its loads
+    // (16 in flight) before using any (the partials are few: latency, not bandwidth, sets this
+    // kernel's time, and every lane of every warp takes part)
+    constexpr int kInFlight = 16;
     const int64_t cpg = group_cols >> 7;
-    const uint32_t *p = partial + (int64_t)blockIdx.x * cpg;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // lanes walk the group's column blocks, warps its 32-row blocks, eight independent loads in
-    // flight per lane (the partials are few: latency, not bandwidth, sets this kernel's time)
+    const uint32_t total = (uint32_t)(rows32 * cpg);        // < 2^31 (checked by the host)
+    const uint32_t ucpg = (uint32_t)cpg;
     uint32_t m = 0;
-    for (int64_t c = lane; c < cpg; c += 32) {
-        for (int64_t r0 = warp; r0 < rows32; r0 += (int64_t)kWarps * kRowsInFlight) {
-            uint32_t v[kRowsInFlight];
+    for (uint32_t f0 = threadIdx.x; f0 < total; f0 += (uint32_t)kThreads * kInFlight) {
+        uint32_t v[kInFlight];
 #pragma unroll
-            for (int u = 0; u < kRowsInFlight; ++u) {
-                const int64_t r = r0 + (int64_t)u * kWarps;
-                v[u] = r < rows32 && NVFP4_CHECKED((int64_t)blockIdx.x * cpg + r * n128 + c, 1, rows32 * n128, status)
-                           ? p[r * n128 + c] : 0u;
-            }
-#pragma unroll
-            for (int u = 0; u < kRowsInFlight; ++u) m = max(m, v[u]);
+        for (int u = 0; u < kInFlight; ++u) {
+            const uint32_t f = f0 + (uint32_t)u * kThreads;
+            const uint32_t r = f / ucpg, c = f - r * ucpg;
+            const int64_t idx = (int64_t)r * n128 + (int64_t)blockIdx.x * cpg + c;
+            v[u] = f < total && NVFP4_CHECKED(idx, 1, rows32 * n128, status) ? partial[idx] : 0u;
         }
+#pragma unroll
+        for (int u = 0; u < kInFlight; ++u) m = max(m, v[u]);
     }
     m = warp_max(m);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
