@@ -54,3 +54,25 @@ def test_op_summary_excludes_the_side_stream_op():
     # 8.8e8 B in 0.14 ms = 6285.7 GB/s; 2.65e11 FLOP in 0.1 ms = 2650 TFLOP/s
     assert k["deq"]["us_per_launch"] == 140.0 and abs(k["deq"]["achieved"] - 6285.7) < 0.1
     assert k["gemm"]["unit"] == "TFLOP/s" and abs(k["gemm"]["frac"] - 2650 / 5500) < 1e-4
+
+
+def test_profiled_traffic_is_used_only_for_matching_sources(tmp_path, monkeypatch):
+    # the roofline's `traffic` comes from a committed ncu summary only while the kernel sources
+    # it names hash to the digest recorded with the capture
+    csrc = tmp_path / "bit_kv_cache_24_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("kernel v1")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    digest = bench.kernel_source_digest(["k.cu"])
+    (tmp_path / "profiles" / "k_case.md").write_text(
+        f"# k\n\n- kernel_source_digest: `{digest}`\n- dram_bytes_per_launch: `123456`\n")
+    assert bench.profiled_traffic("k_case", digest) == 123456.0
+    (csrc / "k.cu").write_text("kernel v2")            # the kernel changed after the capture
+    assert bench.profiled_traffic("k_case", bench.kernel_source_digest(["k.cu"])) is None
+    assert bench.profiled_traffic("missing_case", digest) is None
+
+
+def test_attention_slots_option():
+    assert bench.parse_args([]).attn_slots == bench.SLOTS
+    assert bench.parse_args(["--op", "attention", "--attn-slots", "1"]).attn_slots == 1
