@@ -205,7 +205,9 @@ NVFP4_API nvfp4_status nvfp4_gemm_quant_out(const nvfp4_tensor *A, const nvfp4_t
  * max |Y[:, g*group_cols : (g+1)*group_cols]|, exact (a max of the stored BF16 values), e.g. the
  * amax of the K and V slices of a fused QKV projection.  Requires group_cols % 256 == 0,
  * N % group_cols == 0, and ws of nvfp4_gemm_colamax_workspace(M, N) bytes (per-block partial
- * maxima; no initialisation needed).  inf/NaN in a group sets NVFP4_ERR_NONFINITE and stores NaN.
+ * maxima; no initialisation needed); NVFP4_ERR_UNSUPPORTED when a group holds 2^31 or more of
+ * those partials (ceil(M / 32) * group_cols / 128).  inf/NaN in a group sets NVFP4_ERR_NONFINITE
+ * and stores NaN.
  */
 NVFP4_API size_t nvfp4_gemm_colamax_workspace(int64_t M, int64_t N);
 NVFP4_API nvfp4_status nvfp4_gemm_colamax(const nvfp4_tensor *A, const nvfp4_tensor *B, const void *bias_bf16,
